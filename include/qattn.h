@@ -1,0 +1,185 @@
+/*
+ * qattn.h — C ABI of the B200 (sm_100a) quantized attention prefill library.
+ *
+ * The operation is the SageAttention-style INT8-QK / FP8-PV non-causal
+ * attention whose numerics the page "Exact Numerical Contract" fixes:
+ *   prep   : per-head Q/K RMSNorm + split-half RoPE        ("Preparation")
+ *   quant  : exact K mean subtraction, INT8 Q (32-row groups), INT8 K (64-row
+ *            blocks), FP8 E4M3 V with per-channel scales   ("Preparation" step 4,
+ *            "Q And K Quantization", "V And PV")
+ *   fwd    : INT8 QK^T, base-2 online softmax over 64-key tiles in order, FP8
+ *            P.V, BF16 NHD output                          ("INT8 QK And Score
+ *            Domain", "Online Softmax", "V And PV", "Finalization And Tails")
+ * plus the per-head Walsh-Hadamard rotated int8-K variant of the page
+ * "npu plan P7: int8 KV with per-head Hadamard rotation" (design note; PR #1273).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers marked (device) must point to device memory of the current CUDA
+ *     device; the caller allocates and owns every buffer.  The library keeps no
+ *     state between calls except one thread-local error string.
+ *   - Calls are stream-ordered and asynchronous on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream).  Argument errors are reported synchronously
+ *     and launch nothing.  A failed launch returns QATTN_ERR_CUDA.  A device-side
+ *     bounded wait that gave up is reported through the caller's `dev_err` word
+ *     (read it with qattn_check after the stream finishes).
+ *   - BF16 is passed as uint16_t bit patterns, FP8 E4M3 as uint8_t, FP16 as
+ *     uint16_t.  Inputs are finite; NaN/Inf behaviour is not part of the contract.
+ *   - No entry point falls back to another implementation: an unsupported case
+ *     returns a named refusal (the refusal convention of the "npu plan P7" page).
+ */
+#ifndef QATTN_H_
+#define QATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QATTN_OK = 0,
+  QATTN_ERR_NULL = 1,        /* a required pointer is NULL                         */
+  QATTN_ERR_SHAPE = 2,       /* a size is <= 0, too large, or inconsistent         */
+  QATTN_ERR_STRIDE = 3,      /* last stride != 1, or a row / base not 16-B aligned */
+  QATTN_ERR_UNSUPPORTED = 4, /* D not in {64,128,256}, bad rotary_dim, Hq % Hkv,
+                                bad k_scale_mode, or a device that is not sm_100   */
+  QATTN_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the query says      */
+  QATTN_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed                  */
+  QATTN_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up (via dev_err)   */
+} qattn_status;
+
+/* A strided BF16 view of logical shape [B, N, H, D].  stride[] are ELEMENT
+ * strides of the four logical dims; stride[3] must be 1 and stride[0..2] and the
+ * base address must keep every (b, n, h) row 16-byte aligned.  The canonical
+ * interleaved QKV buffer of the "Canonical Boundary" section is three such views
+ * of one [N, 21504] buffer at element offsets 0 / 7168 / 14336 with strides
+ * {813066240, 21504, 128, 1}. */
+typedef struct {
+  const void* ptr;  /* (device) BF16 data */
+  int64_t stride[4];
+} qattn_bnhd;
+
+/* ---------------------------------------------------------------- prep
+ * Per-head RMSNorm then split-half RoPE on Q [B,N,Hq,D] and K [B,N,Hkv,D]
+ * ("Exact Numerical Contract", "Preparation" steps 1-3).
+ *   r   = 1/sqrt(mean(x^2) + eps), FP32 with IEEE sqrt/divide; the sum of squares
+ *         is taken as D/8 lanes of 8 consecutive dims (left to right) then an XOR
+ *         butterfly over lanes (D/16, ..., 2, 1)
+ *   n   = bf16_rn(x*r);  y = bf16_rn(n * weight[d])   (weight [D], all heads)
+ *   RoPE on dims [0, rotary_dim): pairs (i, i+R/2) with BF16 coefficients
+ *         cos/sin(pos * theta^(-2i/R)) computed in FP64 and rounded once to BF16;
+ *         y_i' = bf16_rn(y_i c - y_{i+R/2} s), y_{i+R/2}' = bf16_rn(y_{i+R/2} c + y_i s)
+ *   pos = pos_offset + n.
+ * Arguments
+ *   q, k            strided BF16 inputs (device)
+ *   q_weight, k_weight  BF16 [D] (device); NULL skips the norm of that tensor
+ *   rotary_dim      0 (no RoPE) or a multiple of 16 with rotary_dim <= D
+ *   q_out, k_out    contiguous BF16 [B,N,Hq,D] / [B,N,Hkv,D] (device)
+ * D in {64,128,256}.  Errors: NULL, SHAPE, STRIDE, UNSUPPORTED, CUDA. */
+qattn_status qattn_prep(int B, int N, int Hq, int Hkv, int D,
+                        qattn_bnhd q, qattn_bnhd k,
+                        const uint16_t* q_weight, const uint16_t* k_weight, float eps,
+                        int rotary_dim, double rope_theta, int64_t pos_offset,
+                        uint16_t* q_out, uint16_t* k_out, void* stream);
+
+/* ---------------------------------------------------------------- quant
+ * Bytes of device workspace qattn_quant / qattn_quant_hadamard need for a KV
+ * sequence of Nkv rows: FP64 K column partials per 64-row block, FP32 V column
+ * maxima per block and the FP32 V factors.  Returns 0 on invalid sizes. */
+size_t qattn_quant_workspace_bytes(int B, int Nkv, int Hkv, int D);
+
+/* Quantize prepared Q/K and raw V ("Preparation" step 4, "Q And K Quantization",
+ * "V And PV").
+ *   k_mean[b,h,d] = (float)( sum_j sum_{r in block j} k_r / N ), FP64, rows then
+ *                   blocks ascending
+ *   K: x = (float)k - k_mean (FP32); one scale per 64 rows; Q: one scale per 32
+ *   rows inside 128-row tiles, G = 4*ceil(Nq/128) scales per (b,h):
+ *       amax = max(1e-7f, max|x|); scale = amax/127.0f; q8 = rni_sat_s8(x*(127.0f/amax))
+ *   (tail rows do not count; groups with no row get 1e-7f/127.0f)
+ *   V: amax = max(1e-7f, max_n |v|) per (b,h,d); v_scale = amax/2.25f;
+ *       v8 = e4m3_rn_satfinite(v * (2.25f/amax)), stored dim-major.
+ * Arguments (all device)
+ *   qp [B,Nq,Hq,D], kp [B,Nkv,Hkv,D], v [B,Nkv,Hkv,D]  strided BF16 views
+ *   q8      int8 [B,Hq,Nq,D]            q_scale FP32 [B,Hq,4*ceil(Nq/128)]
+ *   k8      int8 [B,Hkv,Nkv,D]          k_scale FP32 [B,Hkv,ceil(Nkv/64)]
+ *   k_mean  FP32 [B,Hkv,D]
+ *   v8t     E4M3 [B,Hkv,D,64*ceil(Nkv/64)] (keys contiguous; rows >= Nkv are 0)
+ *   v_scale FP32 [B,Hkv,D]
+ *   workspace, workspace_bytes: >= qattn_quant_workspace_bytes(B,Nkv,Hkv,D)
+ * Hq % Hkv == 0.  Errors: NULL, SHAPE, STRIDE, UNSUPPORTED, WORKSPACE, CUDA. */
+qattn_status qattn_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                         qattn_bnhd qp, qattn_bnhd kp, qattn_bnhd v,
+                         int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                         float* k_mean, uint8_t* v8t, float* v_scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Hadamard-rotated variant ("npu plan P7" page: rotate Q and K by the same
+ * per-head Walsh-Hadamard H, store K int8 with one FP16 scale per (head, token)).
+ *   x' = FWHT(x) / sqrt(D) in FP32 (Sylvester order, no sign vector; stages
+ *        h = 1, 2, ..., D/2 mapping (a, b) -> (a+b, a-b)); D in {64, 256}
+ *   Q': INT8 per 32-row group as qattn_quant;  no K mean
+ *   K': amax = max(1e-7f, max_d |k'|) per token; k_scale_f16 = fp16_rn(amax/127.0f);
+ *       k8 = rni_sat_s8(k' * (127.0f/amax))
+ *   V : as qattn_quant.
+ * k_scale_f16 is FP16 [B,Hkv,Nkv] (device).  Use qattn_fwd with k_scale_mode 1.
+ * Errors: as qattn_quant. */
+qattn_status qattn_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                                  qattn_bnhd q, qattn_bnhd k, qattn_bnhd v,
+                                  int8_t* q8, float* q_scale, int8_t* k8,
+                                  uint16_t* k_scale_f16, uint8_t* v8t, float* v_scale,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- fwd
+ * Fused attention ("INT8 QK And Score Domain", "Online Softmax", "V And PV",
+ * "Finalization And Tails").  Per query row, over 64-key tiles t = 0, 1, ... in
+ * order, with m = -5e6f, d = 1.0f, O = 0 initially:
+ *   s_j  = ((float)S_j * (q_scale * k_scale_j)) * c, c = log2(e) * sm_scale,
+ *          S = Q8 K8^T exact in INT32; keys >= Nkv get -5e6f
+ *   mn   = max(m, max_j s_j - 8.807f); old = 2^(m - mn); d *= old; O *= old
+ *   p_j  = 2^(s_j - mn); d += p_j (FP32, unquantized); P8 = e4m3_rn_satfinite(p)
+ *   O   += P8 . V8 (tcgen05 FP8 MMA, FP32 accumulation in tensor memory)
+ *   out  = bf16_rn(O / d * v_scale[d]), query rows < Nq only.
+ * Arguments (all device except scalars)
+ *   q8, q_scale, k8, v8t, v_scale  as produced by qattn_quant / _hadamard
+ *   k_scale       k_scale_mode 0: FP32 [B,Hkv,ceil(Nkv/64)];
+ *                 k_scale_mode 1: FP16 [B,Hkv,Nkv] (per token)
+ *   sm_scale      softmax scale; 0 means 1/sqrt(D)
+ *   out           contiguous BF16 [B,Nq,Hq,D]
+ *   dev_err       one int32 (device), caller-owned; the kernel ORs error bits into
+ *                 it (0 = success); read it with qattn_check.
+ * D in {64,128,256}; Hq % Hkv == 0; GQA head h reads KV head h / (Hq/Hkv).
+ * Errors: NULL, SHAPE, UNSUPPORTED, CUDA (synchronous); TIMEOUT (via dev_err). */
+qattn_status qattn_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                       const int8_t* q8, const float* q_scale,
+                       const int8_t* k8, const void* k_scale, int k_scale_mode,
+                       const uint8_t* v8t, const float* v_scale, float sm_scale,
+                       uint16_t* out, int* dev_err, void* stream);
+
+/* Raw INT32 score tiles S = Q8 K8^T through the same TMA + tcgen05 INT8 path as
+ * qattn_fwd ("INT8 QK And Score Domain"), for bit-exact checks.
+ *   tiles    int32 [n_tiles][4] = (b, h, q_tile, k_tile) (device); q_tile indexes
+ *            128-row query tiles, k_tile 64-row key tiles; rows past Nq/Nkv read 0
+ *   s_out    int32 [n_tiles][128][64] (device)
+ * Errors: NULL, SHAPE, UNSUPPORTED, CUDA; TIMEOUT via dev_err. */
+qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                          const int8_t* q8, const int8_t* k8,
+                          const int32_t* tiles, int n_tiles, int32_t* s_out,
+                          int* dev_err, void* stream);
+
+/* ---------------------------------------------------------------- status
+ * Synchronize `stream`, read the device error word and map it: 0 -> QATTN_OK,
+ * a timed-out wait -> QATTN_ERR_TIMEOUT; a CUDA error -> QATTN_ERR_CUDA. */
+qattn_status qattn_check(const int* dev_err, void* stream);
+
+/* Human-readable reason of the last non-OK status returned on this thread. */
+const char* qattn_last_error(void);
+
+/* Library version string. */
+const char* qattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QATTN_H_ */

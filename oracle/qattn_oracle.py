@@ -55,18 +55,22 @@ def ceil_div(a: int, b: int) -> int:
 
 
 # ============================================================ preparation
-def rope_tables(n_pos: int, rotary_dim: int, theta: float, pos_offset: int = 0):
+def rope_tables(n_pos: int, rotary_dim: int, theta: float, pos_offset: int = 0,
+                positions=None):
     """BF16 cos/sin coefficients for split-half RoPE ("Preparation" step 3).
 
     Reading (the page says only "BF16 coefficients"): frequency
     ``theta^(-(2i)/R)`` for pair i < R/2, angle ``pos * freq``, cos and sin,
-    all in FP64, each rounded once to BF16 RN.  Returns two uint16 arrays of
-    shape [n_pos, R/2].
+    all in FP64, each rounded once to BF16 RN.  Positions are
+    ``pos_offset + 0..n_pos-1`` unless ``positions`` lists them.  Returns two
+    uint16 arrays of shape [n_pos, R/2].
     """
     half = rotary_dim // 2
     i = np.arange(half, dtype=np.float64)
     inv_freq = np.power(np.float64(theta), -(2.0 * i) / np.float64(rotary_dim))
-    pos = (np.arange(n_pos, dtype=np.int64) + pos_offset).astype(np.float64)
+    if positions is None:
+        positions = np.arange(n_pos, dtype=np.int64) + pos_offset
+    pos = np.asarray(positions, dtype=np.int64).astype(np.float64)
     ang = pos[:, None] * inv_freq[None, :]
     return bf16_bits_from_f64(np.cos(ang)), bf16_bits_from_f64(np.sin(ang))
 
@@ -95,7 +99,7 @@ def rms_sum_of_squares(x: np.ndarray) -> np.ndarray:
 
 
 def prep(x_bits: np.ndarray, weight_bits, eps: float, rotary_dim: int,
-         theta: float = 10000.0, pos_offset: int = 0) -> np.ndarray:
+         theta: float = 10000.0, pos_offset: int = 0, positions=None) -> np.ndarray:
     """Per-head RMSNorm then split-half RoPE on one BF16 [B,N,H,D] tensor.
 
     "Preparation" steps 1-3:
@@ -109,7 +113,8 @@ def prep(x_bits: np.ndarray, weight_bits, eps: float, rotary_dim: int,
                      y_{i+R/2} = bf16_rn(y_{i+R/2}*c + y_i*s)
       dims >= R pass through.
     ``weight_bits`` None skips the norm (and its weight); ``rotary_dim`` 0
-    skips RoPE.  Positions are ``pos_offset + n``.
+    skips RoPE.  Positions are ``pos_offset + n`` unless ``positions`` gives
+    one per token (for a sample of tokens).
     """
     x = f32_from_bf16_bits(x_bits)
     b, n, h, d = x.shape
@@ -124,7 +129,7 @@ def prep(x_bits: np.ndarray, weight_bits, eps: float, rotary_dim: int,
         y = np.array(x_bits, dtype=np.uint16, copy=True)
     if rotary_dim:
         half = rotary_dim // 2
-        cb, sb = rope_tables(n, rotary_dim, theta, pos_offset)
+        cb, sb = rope_tables(n, rotary_dim, theta, pos_offset, positions)
         c = f32_from_bf16_bits(cb)[None, :, None, :]
         s = f32_from_bf16_bits(sb)[None, :, None, :]
         yf = f32_from_bf16_bits(y)

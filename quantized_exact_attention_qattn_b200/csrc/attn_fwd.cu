@@ -1,0 +1,564 @@
+// attn_fwd.cu — fused INT8-QK / FP8-PV attention mainloop for sm_100a.
+//
+// Numerics: "Exact Numerical Contract", sections "INT8 QK And Score Domain",
+// "Online Softmax", "V And PV", "Finalization And Tails".  Per query row and
+// per 64-key tile t (ascending):
+//   s = ((float)S * (q_scale * k_scale)) * c        S = Q8 K8^T (exact INT32)
+//   mn = max(m, max(s) - 8.807);  old = ex2(m - mn);  d *= old;  O *= old
+//   p = ex2(s - mn);  d += p;  P8 = e4m3(p);  O += P8 V8;  m = mn
+//   out = bf16(O * rcp(d) * v_scale)
+//
+// Blackwell mapping (one CTA = NQT query tiles of 128 rows of one (b, h)):
+//   warp 0      TMA producer: Q tiles once, then K/V tiles into a STAGES ring
+//   warp 1      tensor-memory owner and single-thread tcgen05.mma issuer:
+//               QK^T as kind::i8 (M=128, N=64, K=32 steps) into TMEM S[i],
+//               P.V as kind::f8f6f4 with P read from TMEM (M=128, N=D, K=32)
+//               accumulating into TMEM O[i]
+//   warps 4..   one 128-thread softmax warpgroup per query tile; thread r owns
+//               query row r (TMEM lane r): tcgen05.ld of its 64 scores, the
+//               online-softmax update, the O rescale (only when a row's max
+//               moved), tcgen05.st of its 64 FP8 probabilities, and the final
+//               normalisation + BF16 store.
+// The MMA warp issues PV(i, t) then QK(i, t+1) per tile i, so while one
+// warpgroup runs the softmax of tile t the tensor core works for the other.
+// Every wait is bounded; a timeout sets a device error bit and all roles drain.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "qattn_device.cuh"
+#include "qattn_internal.h"
+
+namespace qattn {
+namespace {
+
+constexpr int BM = 128;   // query rows per tile (TMEM lanes)
+constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
+constexpr float kMInit = -5000000.0f;
+constexpr float kFp8Offset = 8.807f;
+constexpr float kMasked = -5000000.0f;
+
+template <int D, int NQT>
+struct Cfg {
+  static constexpr int STAGES = (D == 256) ? 3 : 4;
+  static constexpr int KCH = (D >= 128) ? 128 : 64;       // K-major swizzle row width (bytes)
+  static constexpr int NCH = D / KCH;                      // 128-byte column chunks per row
+  static constexpr uint32_t SW_QK = (KCH == 128) ? 2u : 4u; // 128B or 64B swizzle
+  static constexpr int Q_BYTES = BM * D;
+  static constexpr int K_BYTES = BN * D;
+  static constexpr int V_BYTES = D * BN;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_K = SMEM_Q + NQT * Q_BYTES;
+  static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
+  static constexpr int SMEM_BAR = SMEM_V + STAGES * V_BYTES;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NQT + 1;
+  static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
+  static constexpr int THREADS = 128 + 128 * NQT;
+  static constexpr uint32_t O_COL = 0;
+  static constexpr uint32_t S_COL = NQT * D;
+  static constexpr uint32_t P_COL = S_COL + NQT * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(P_COL + NQT * (BN / 4) <= TMEM_COLS, "tensor memory budget");
+  static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
+  static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
+};
+
+struct FwdParams {
+  const float* q_scale;
+  const void* k_scale;
+  const float* v_scale;
+  uint16_t* out;
+  int* dev_err;
+  int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups, k_scale_mode;
+  float c;
+};
+
+template <int D, int NQT>
+__global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = Cfg<D, NQT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + C::STAGES;
+  uint64_t* s_full = kv_empty + C::STAGES;
+  uint64_t* p_full = s_full + NQT;
+  uint64_t* o_done = p_full + NQT;
+  uint64_t* drain = o_done + NQT;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (b, h, group of NQT query tiles), tiles of one head adjacent
+  const int item = blockIdx.x;
+  const int grp = item % p.n_groups;
+  const int bh = item / p.n_groups;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
+  const int hkv = h / (p.Hq / p.Hkv);
+  const int bhkv = b * p.Hkv + hkv;
+  const int qt0 = grp * NQT;
+  const int nvalid = min(NQT, p.nQ - qt0);
+  const int nK = p.nK;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int i = 0; i < NQT; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 4);
+      mbar_init(o_done + i, 1);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort = &abort_flag;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nvalid * C::Q_BYTES));
+      for (int i = 0; i < nvalid; ++i)
+        for (int ch = 0; ch < C::NCH; ++ch)
+          tma_load_3d(smem + C::SMEM_Q + i * C::Q_BYTES + ch * (BM * C::KCH), &tmQ, q_full,
+                      ch * C::KCH, (qt0 + i) * BM, bh);
+      int issued = 0;
+      for (int t = 0; t < nK; ++t) {
+        const int s = t % C::STAGES;
+        if (t >= C::STAGES &&
+            !mbar_wait(kv_empty + s, ((t / C::STAGES) - 1) & 1, abort, p.dev_err, kErrTimeoutKV))
+          break;
+        mbar_arrive_expect_tx(kv_full + s, static_cast<uint32_t>(C::K_BYTES + C::V_BYTES));
+        for (int ch = 0; ch < C::NCH; ++ch)
+          tma_load_3d(smem + C::SMEM_K + s * C::K_BYTES + ch * (BN * C::KCH), &tmK, kv_full + s,
+                      ch * C::KCH, t * BN, bhkv);
+        tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN, 0, bhkv);
+        issued = t + 1;
+      }
+      // drain: every issued copy must land before the CTA may exit
+      int dummy = 0;
+      mbar_wait(q_full, 0, &dummy, p.dev_err, kErrTimeoutDrain);
+      for (int u = max(0, issued - C::STAGES); u < issued; ++u)
+        mbar_wait(kv_full + (u % C::STAGES), (u / C::STAGES) & 1, &dummy, p.dev_err,
+                  kErrTimeoutDrain);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+      const uint32_t sK = smem_u32(smem + C::SMEM_K);
+      const uint32_t sV = smem_u32(smem + C::SMEM_V);
+      auto issue_qk = [&](int i, int s) {
+        const uint32_t d_tm = tmem + C::S_COL + i * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
+          const uint64_t ad = smem_desc(sQ + i * C::Q_BYTES + ch * (BM * C::KCH) + off,
+                                        8 * C::KCH, C::SW_QK);
+          const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
+                                        8 * C::KCH, C::SW_QK);
+          mma_i8_ss(d_tm, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full + i);
+      };
+      auto issue_pv = [&](int i, int s, int t) {
+        const uint32_t d_tm = tmem + C::O_COL + i * D;
+        const uint32_t a_tm = tmem + C::P_COL + i * (BN / 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 32; ++kk) {
+          const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
+          mma_f8_ts(d_tm, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(o_done + i);
+      };
+      bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ);
+      if (ok) ok = mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < nvalid; ++i) issue_qk(i, 0);
+      }
+      for (int t = 0; ok && t < nK; ++t) {
+        const int s = t % C::STAGES;
+        const int s1 = (t + 1) % C::STAGES;
+        bool next_ready = false;
+        for (int i = 0; ok && i < nvalid; ++i) {
+          ok = mbar_wait(p_full + i, t & 1, abort, p.dev_err, kErrTimeoutP);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(i, s, t);
+          if (t + 1 < nK) {
+            if (!next_ready) {
+              ok = mbar_wait(kv_full + s1, ((t + 1) / C::STAGES) & 1, abort, p.dev_err,
+                             kErrTimeoutKV);
+              if (!ok) break;
+              tc_fence_after();
+              next_ready = true;
+            }
+            issue_qk(i, s1);
+          }
+        }
+        if (ok) tc_commit(kv_empty + s);
+      }
+      // drain: wait for every issued tensor-core operation before tear-down
+      tc_commit(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, &dummy, p.dev_err, kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ================================================================ softmax
+    const int wg = (warp - 4) >> 2;
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    if (wg < nvalid) {
+      const int qt = qt0 + wg;
+      const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+      const uint32_t tS = tmem + lane_off + C::S_COL + wg * BN;
+      const uint32_t tP = tmem + lane_off + C::P_COL + wg * (BN / 4);
+      const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
+      const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
+      const int last_valid = p.Nkv - (nK - 1) * BN;
+      float m = kMInit, den = 1.0f;
+      bool ok = true;
+      for (int t = 0; t < nK; ++t) {
+        if (!mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sraw[64];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+        tmem_wait_ld();
+        float sv[64];
+        if (p.k_scale_mode == 0) {
+          const float ks = static_cast<const float*>(p.k_scale)[static_cast<int64_t>(bhkv) * nK + t];
+          const float alpha = __fmul_rn(qs, ks);
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            sv[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(sraw[j])), alpha), p.c);
+        } else {
+          const __half* ks16 = static_cast<const __half*>(p.k_scale) +
+                               static_cast<int64_t>(bhkv) * p.Nkv + t * BN;
+          const int nv = (t == nK - 1) ? last_valid : BN;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float ks = (j < nv) ? __half2float(ks16[j]) : 0.0f;
+            sv[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(sraw[j])),
+                                        __fmul_rn(qs, ks)), p.c);
+          }
+        }
+        if (t == nK - 1) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (j >= last_valid) sv[j] = kMasked;
+        }
+        float mx = sv[0];
+#pragma unroll
+        for (int j = 1; j < 64; ++j) mx = fmaxf(mx, sv[j]);
+        const float mn = fmaxf(m, __fsub_rn(mx, kFp8Offset));
+        const float old = ex2_approx(__fsub_rn(m, mn));
+        den = __fmul_rn(den, old);
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 64; j += 4) {
+          const float p0 = ex2_approx(__fsub_rn(sv[j], mn));
+          const float p1 = ex2_approx(__fsub_rn(sv[j + 1], mn));
+          const float p2 = ex2_approx(__fsub_rn(sv[j + 2], mn));
+          const float p3 = ex2_approx(__fsub_rn(sv[j + 3], mn));
+          den = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(den, p0), p1), p2), p3);
+          pk[j / 4] = static_cast<uint32_t>(cvt_e4m3x2(p0, p1)) |
+                      (static_cast<uint32_t>(cvt_e4m3x2(p2, p3)) << 16);
+        }
+        if (t > 0) {
+          // PV(t-1) must be finished: it reads P and accumulates into O
+          if (!mbar_wait(o_done + wg, (t - 1) & 1, abort, p.dev_err, kErrTimeoutO)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, old != 1.0f)) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__fmul_rn(__uint_as_float(o[j]), old));
+              tmem_st32(tO + c0, o);
+            }
+          }
+        }
+        tmem_st16(tP, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + wg);
+        m = mn;
+      }
+      // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only
+      if (ok && mbar_wait(o_done + wg, (nK - 1) & 1, abort, p.dev_err, kErrTimeoutO)) {
+        tc_fence_after();
+        const float inv = rcp_approx(den);
+        const int n = qt * BM + row;
+        const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
+        uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld();
+          if (n < p.Nq) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float a0 = __fmul_rn(__fmul_rn(__uint_as_float(o[j]), inv), vs[c0 + j]);
+              const float a1 = __fmul_rn(__fmul_rn(__uint_as_float(o[j + 1]), inv), vs[c0 + j + 1]);
+              w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a0))) |
+                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a1))) << 16);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+            d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ scores (debug)
+// One CTA per requested (b, h, q_tile, k_tile): TMA both tiles, the same
+// kind::i8 MMA sequence as the mainloop, tcgen05.ld of the INT32 tile.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const int32_t* tiles, int32_t* s_out, int Hq, int Hkv, int* dev_err) {
+  using C = Cfg<D, 1>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + C::Q_BYTES;
+  __shared__ uint64_t bar_ld, bar_mma;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* tl = tiles + 4 * blockIdx.x;
+  const int b = tl[0], h = tl[1], qt = tl[2], kt = tl[3];
+  const int hkv = h / (Hq / Hkv);
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_ld, 1);
+    mbar_init(&bar_mma, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort = &abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar_ld, static_cast<uint32_t>(C::Q_BYTES + C::K_BYTES));
+    for (int ch = 0; ch < C::NCH; ++ch) {
+      tma_load_3d(sQ + ch * (BM * C::KCH), &tmQ, &bar_ld, ch * C::KCH, qt * BM, b * Hq + h);
+      tma_load_3d(sK + ch * (BN * C::KCH), &tmK, &bar_ld, ch * C::KCH, kt * BN, b * Hkv + hkv);
+    }
+  }
+  if (threadIdx.x == 32) {
+    int dummy = 0;
+    if (mbar_wait(&bar_ld, 0, abort, dev_err, kErrTimeoutQ)) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk) {
+        const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
+        const uint64_t ad = smem_desc(smem_u32(sQ) + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
+        const uint64_t bd = smem_desc(smem_u32(sK) + ch * (BN * C::KCH) + off, 8 * C::KCH, C::SW_QK);
+        mma_i8_ss(tmem, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(&bar_mma);
+    (void)dummy;
+  }
+  __syncwarp();
+  bool ok = mbar_wait(&bar_mma, 0, abort, dev_err, kErrTimeoutS);
+  {
+    int dummy = 0;   // the TMA must have landed before exit, whatever happened
+    if (threadIdx.x == 0) mbar_wait(&bar_ld, 0, &dummy, dev_err, kErrTimeoutDrain);
+  }
+  if (ok) {
+    tc_fence_after();
+    uint32_t r[64];
+    const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    tmem_wait_ld();
+    int4* dst = reinterpret_cast<int4*>(s_out + (static_cast<int64_t>(blockIdx.x) * BM + warp * 32 + lane) * BN);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      dst[j] = make_int4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D uint8 tensor map: dims {inner, rows, planes}, row pitch = inner bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, rows, planes};
+  const cuuint64_t strides[2] = {inner, inner * rows};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NQT>
+cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
+                         const float* q_scale, const int8_t* k8, const void* k_scale,
+                         int k_scale_mode, const uint8_t* v8t, const float* v_scale, float c,
+                         uint16_t* out, int* dev_err, cudaStream_t st, const char** why) {
+  using Cf = Cfg<D, NQT>;
+  const int nQ = (Nq + BM - 1) / BM;
+  const int nK = (Nkv + BN - 1) / BN;
+  const CUtensorMapSwizzle swqk =
+      (Cf::KCH == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap mQ, mK, mV;
+  if (!make_map(&mQ, q8, D, Nq, static_cast<uint64_t>(B) * Hq, Cf::KCH, BM, swqk) ||
+      !make_map(&mK, k8, D, Nkv, static_cast<uint64_t>(B) * Hkv, Cf::KCH, BN, swqk) ||
+      !make_map(&mV, v8t, static_cast<uint64_t>(nK) * BN, D, static_cast<uint64_t>(B) * Hkv, BN, D,
+                CU_TENSOR_MAP_SWIZZLE_64B)) {
+    *why = "cuTensorMapEncodeTiled failed (pointer alignment or size)";
+    return cudaErrorInvalidValue;
+  }
+  FwdParams p{};
+  p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale; p.out = out; p.dev_err = dev_err;
+  p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
+  p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
+  p.k_scale_mode = k_scale_mode; p.c = c;
+  // at least 116 KB so that one CTA (and one 512-column TMEM allocation) owns an SM
+  const int smem = (Cf::SMEM_BYTES + 1024 > 116 * 1024) ? Cf::SMEM_BYTES + 1024 : 116 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(B) * Hq * p.n_groups);
+  attn_fwd_kernel<D, NQT><<<grid, Cf::THREADS, smem, st>>>(mQ, mK, mV, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_scores_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
+                            const int8_t* k8, const int32_t* tiles, int n_tiles, int32_t* s_out,
+                            int* dev_err, cudaStream_t st, const char** why) {
+  using Cf = Cfg<D, 1>;
+  const CUtensorMapSwizzle swqk =
+      (Cf::KCH == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap mQ, mK;
+  if (!make_map(&mQ, q8, D, Nq, static_cast<uint64_t>(B) * Hq, Cf::KCH, BM, swqk) ||
+      !make_map(&mK, k8, D, Nkv, static_cast<uint64_t>(B) * Hkv, Cf::KCH, BN, swqk)) {
+    *why = "cuTensorMapEncodeTiled failed (pointer alignment or size)";
+    return cudaErrorInvalidValue;
+  }
+  const int smem = Cf::Q_BYTES + Cf::K_BYTES + 1024;
+  cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  scores_kernel<D><<<n_tiles, 128, smem, st>>>(mQ, mK, tiles, s_out, Hq, Hkv, dev_err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
+                       const float* q_scale, const int8_t* k8, const void* k_scale,
+                       int k_scale_mode, const uint8_t* v8t, const float* v_scale,
+                       float score_c, uint16_t* out, int* dev_err, cudaStream_t st,
+                       const char** why) {
+  switch (D) {
+    case 64:
+      return launch_fwd_t<64, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
+                                 v_scale, score_c, out, dev_err, st, why);
+    case 128:
+      return launch_fwd_t<128, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
+                                  v8t, v_scale, score_c, out, dev_err, st, why);
+    case 256:
+      return launch_fwd_t<256, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
+                                  v8t, v_scale, score_c, out, dev_err, st, why);
+    default:
+      *why = "head dimension must be 64, 128 or 256";
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
+                          const int8_t* k8, const int32_t* tiles, int n_tiles, int32_t* s_out,
+                          int* dev_err, cudaStream_t st, const char** why) {
+  switch (D) {
+    case 64: return launch_scores_t<64>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
+    case 128: return launch_scores_t<128>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
+    case 256: return launch_scores_t<256>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
+    default:
+      *why = "head dimension must be 64, 128 or 256";
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qattn

@@ -1,0 +1,393 @@
+"""Benchmark of the quantized attention prefill path on B200.
+
+One step = the whole hot path on the canonical call of the "Exact Numerical
+Contract" page: B=1, N=37,810, H=56, D=128, interleaved BF16 QKV [N, 21504]:
+  qattn_prep (RMSNorm + RoPE) -> qattn_quant (K mean, INT8 Q/K, FP8 V)
+  -> qattn_fwd (tcgen05 INT8 QK^T, online softmax, FP8 P.V, BF16 out).
+Value = effective TFLOP/s = 4*B*H*N^2*D per step (all ranks) / step time
+(max over ranks).  Each rank runs its own independent problem (weak scaling,
+no data-path collective).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the CPU oracle (the plain reference implementation of
+the method written for this repository) on a bounded sample of the same
+workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and effective TFLOPS at N=37810 H=56 D=128; % of INT8/FP8 tensor peak"
+WORKLOAD = {"workload": "canonical interleaved-QKV quantized attention prefill",
+            "B": 1, "N": 37810, "H": 56, "D": 128, "qkv_row_width": 21504,
+            "rotary_dim": 96, "causal": False,
+            "l2": "inputs larger than L2 (1.63 GB QKV, 126 MB L2); no flush needed"}
+NOMINAL_FP8_OVER_BF16 = 2.0          # 4.5 / 2.25 PFLOP/s dense (nominal ratio)
+SPEC_FP8_TFLOPS = 4500.0
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 rank if absent)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """Largest value of x over all ranks (x itself with one rank)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def shard_heads(H: int, world: int, rank: int):
+    """Contiguous head range of `rank` when H heads are split over `world`
+    ranks (every head is an independent problem: no exchange is needed)."""
+    base, rem = divmod(H, world)
+    h0 = rank * base + min(rank, rem)
+    return h0, h0 + base + (1 if rank < rem else 0)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+def make_workload(name: str):
+    from quantized_exact_attention_qattn_b200 import synth
+    if name == "profile16k":   # B1 N16384 H32 D128: > L2 inputs, small enough to profile
+        return synth.custom(16, 1, 16384, 32, 128, name="profile16k")
+    return synth.make(name)
+
+
+def workload_config(w) -> dict:
+    if w.name == "canonical":
+        return dict(WORKLOAD)
+    return {"workload": f"{w.name} quantized attention prefill", "B": w.B, "Nq": w.Nq,
+            "Nkv": w.Nkv, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "hadamard": w.hadamard}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(w, heads, q_tiles):
+    """Run the CPU oracle on `heads` x `q_tiles` of workload `w` (all keys).
+    Returns (seconds, attention flops of the sample)."""
+    import numpy as np
+    from oracle import qattn_oracle as O
+    t0 = time.perf_counter()
+    hs = list(heads)
+    rows = np.concatenate([np.arange(128 * t, min(w.Nq, 128 * t + 128)) for t in q_tiles])
+    k = w.k[:, :, hs]
+    v = w.v[:, :, hs]
+    q = w.q[:, rows][:, :, hs]
+    kp = O.prep(k, w.k_weight, w.eps, w.rotary_dim, w.theta)
+    mu = O.k_mean(kp)
+    k8, ks = O.quant_k(kp, mu)
+    v8t, vs = O.quant_v(v)
+    qp = O.prep(q, w.q_weight, w.eps, w.rotary_dim, w.theta, positions=rows)
+    q8, qs = O.quant_q(qp)
+    O.attention(q8, qs, k8, ks, v8t, vs, w.Nkv)
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * len(hs) * len(rows) * w.Nkv * w.D
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_line(w, heads=(0, 1, 2, 3), q_tiles=tuple(range(8))):
+    dt, flops = oracle_sample(w, heads, q_tiles)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": (f"heads {list(heads)} x query tiles {list(q_tiles)} (128 rows each) against "
+                       f"all {w.Nkv} keys, including prep/K-mean/quant of those heads; numpy "
+                       "oracle, BLAS matmul multithreaded, elementwise single-threaded")}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from quantized_exact_attention_qattn_b200 import synth
+    w = synth.make("canonical")
+    times, flops = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, fl = oracle_sample(w, heads=(i % w.Hq,), q_tiles=(i % 296,))
+        if i >= args.warmup:
+            times.append(dt)
+            flops = fl
+    ms = 1e3 * statistics.mean(times)
+    val = flops / (ms / 1e3) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64/f32 (numpy oracle)", "data": "synthetic",
+            "config": dict(WORKLOAD),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": "per step: one head x one 128-row query tile against all "
+                                       "37810 keys, with that head's prep/K-mean/quant"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args):
+    import torch
+    import quantized_exact_attention_qattn_b200 as qa
+    from quantized_exact_attention_qattn_b200 import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+
+    w = make_workload(args.config)
+    if w.qkv is not None:
+        host_qkv = torch.from_numpy(w.qkv).view(torch.bfloat16).pin_memory()
+    else:   # contiguous workloads: one pinned buffer holding q | k | v
+        import numpy as np
+        host_qkv = torch.from_numpy(np.concatenate([w.q.ravel(), w.k.ravel(), w.v.ravel()])
+                                    ).view(torch.bfloat16).pin_memory()
+    qkv = host_qkv.to(dev)
+    if w.qkv is not None:
+        view = qkv.view(w.B, w.Nq, 3, w.Hq, w.D)
+        q, k, v = view[:, :, 0], view[:, :, 1], view[:, :, 2]
+    else:
+        nq, nk = w.q.size, w.k.size
+        q = qkv[:nq].view(w.q.shape)
+        k = qkv[nq:nq + nk].view(w.k.shape)
+        v = qkv[nq + nk:].view(w.v.shape)
+    qw = kw = None
+    if w.q_weight is not None:
+        qw = torch.from_numpy(w.q_weight).view(torch.bfloat16).to(dev)
+        kw = torch.from_numpy(w.k_weight).view(torch.bfloat16).to(dev)
+    pipe = qa.Pipeline(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, hadamard=w.hadamard, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = pipe.attn_ops
+
+    def step(fwd_ev=None):
+        if w.hadamard:
+            pipe.run_quant_hadamard(q, k, v)
+        else:
+            pipe.run_prep(q, k, qw, kw, w.eps, w.rotary_dim, w.theta)
+            pipe.run_quant(pipe.qp, pipe.kp, v)
+        if fwd_ev is not None:
+            fwd_ev[0].record(stream)
+        pipe.run_fwd()
+        if fwd_ev is not None:
+            fwd_ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    pipe.check()
+
+    # ---- device-timed region
+    fwd_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(fwd_events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    pipe.check()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_total, dist, dev)
+    ms_step = ms_total / args.steps
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
+    value = sum_over_ranks(flops, dist, dev) / (ms_step / 1e3) / 1e12
+
+    # ---- end-to-end: pinned host QKV in, host output back, every step
+    out_host = torch.empty(pipe.out.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        qkv.copy_(host_qkv, non_blocking=True)
+        step()
+        out_host.copy_(pipe.out, non_blocking=True)
+
+    e2e_ms = float("nan")
+    if not args.no_e2e:
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
+        pipe.check()
+
+    if rank == 0:
+        peaks = {}
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                peaks = json.load(f)
+        except OSError:
+            pass
+        if "bf16_tflops_sustained" in peaks:
+            peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP8_OVER_BF16
+            peak_src = "measured bf16 sustained x nominal fp8/bf16 ratio 2"
+        else:
+            peak = 1400.0 * NOMINAL_FP8_OVER_BF16
+            peak_src = "fallback bf16 sustained 1.4 PFLOP/s x nominal ratio 2"
+        achieved = flops / (fwd_ms / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 QK / e4m3 PV (f32 accumulate), bf16 in/out", "data": "synthetic",
+            "config": dict(workload_config(w), parallelism=f"{world} independent problems (one per GPU)"),
+            "fwd_ms_per_call": fwd_ms,
+            "fwd_tflops": achieved,
+            "fwd_frac_of_spec_4500": achieved / SPEC_FP8_TFLOPS,
+            "prep_quant_ms": ms_step - fwd_ms,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "attn_fwd_kernel<128,2>",
+                         "peak_source": peak_src,
+                         "algorithmic_work": "4*B*H*N^2*D = %.4e ops per launch" % flops},
+            "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12,
+                    "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": host_qkv.numel() * 2,
+                    "d2h_bytes_per_step": out_host.numel() * 2},
+            "gpu_launches": (3 if w.hadamard else 5) * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline and args.config == "canonical":
+            line["cpu_baseline"] = cpu_baseline_line(w)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--config", default="canonical",
+                    choices=["canonical", "small", "mid", "encoder", "gqa_chunk", "profile16k"],
+                    help="workload; only 'canonical' is the benchmark line, the others are "
+                         "for profiling and checks")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -245,7 +245,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float m = kMInit, den = 1.0f;
       bool ok = true;
       for (int t = 0; t < nK; ++t) {
-        if (!mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS)) { ok = false; break; }
+        // warp-uniform outcome: the tcgen05.ld / shuffles below are warp-collective
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
+        if (!ok) break;
         tc_fence_after();
         uint32_t sraw[64];
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
@@ -293,7 +295,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         if (t > 0) {
           // PV(t-1) must be finished: it reads P and accumulates into O
-          if (!mbar_wait(o_done + wg, (t - 1) & 1, abort, p.dev_err, kErrTimeoutO)) { ok = false; break; }
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(o_done + wg, (t - 1) & 1, abort, p.dev_err, kErrTimeoutO));
+          if (!ok) break;
           tc_fence_after();
           if (__any_sync(0xffffffffu, old != 1.0f)) {
 #pragma unroll 1
@@ -315,7 +319,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m = mn;
       }
       // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only
-      if (ok && mbar_wait(o_done + wg, (nK - 1) & 1, abort, p.dev_err, kErrTimeoutO)) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + wg, (nK - 1) & 1, abort, p.dev_err,
+                                                    kErrTimeoutO));
+      if (ok) {
         tc_fence_after();
         const float inv = rcp_approx(den);
         const int n = qt * BM + row;
@@ -412,7 +418,7 @@ scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     (void)dummy;
   }
   __syncwarp();
-  bool ok = mbar_wait(&bar_mma, 0, abort, dev_err, kErrTimeoutS);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_mma, 0, abort, dev_err, kErrTimeoutS));
   {
     int dummy = 0;   // the TMA must have landed before exit, whatever happened
     if (threadIdx.x == 0) mbar_wait(&bar_ld, 0, &dummy, dev_err, kErrTimeoutDrain);

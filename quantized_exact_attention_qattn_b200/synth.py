@@ -72,17 +72,20 @@ def _normals(rng, shape) -> np.ndarray:
     return rng.standard_normal(shape, dtype=np.float32)
 
 
-def _contig(name, seed, B, N, H, D, k_offset=True, rope=True):
+def _contig(name, seed, B, N, H, D, k_offset=True, rope=True, Hkv=None, Nkv=None):
     rng = np.random.default_rng(seed)
+    Hkv = H if Hkv is None else Hkv
+    Nkv = N if Nkv is None else Nkv
     q = _normals(rng, (B, N, H, D))
-    k = _normals(rng, (B, N, H, D))
-    v = _normals(rng, (B, N, H, D))
+    k = _normals(rng, (B, Nkv, Hkv, D))
+    v = _normals(rng, (B, Nkv, Hkv, D))
     if k_offset:
-        k = k + 2.0 * _normals(rng, (H, D))[None, None]
+        k = k + 2.0 * _normals(rng, (Hkv, D))[None, None]
     qw = 1.0 + 0.1 * _normals(rng, (D,))
     kw = 1.0 + 0.1 * _normals(rng, (D,))
-    return Workload(name, B, N, N, H, H, D, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v),
-                    _bf16_bits(qw), _bf16_bits(kw), 1e-5, 96 if rope else 0, 10000.0, False)
+    return Workload(name, B, N, Nkv, H, Hkv, D, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v),
+                    _bf16_bits(qw), _bf16_bits(kw), 1e-5, 96 if (rope and D >= 96) else 0,
+                    10000.0, False)
 
 
 def _canonical(seed=2, N=37810, H=56, D=128):
@@ -138,6 +141,9 @@ def make(name: str, **overrides) -> Workload:
     raise KeyError(name)
 
 
-def custom(seed, B, N, H, D, *, k_offset=True, rope=True, name="custom") -> Workload:
-    """A contiguous workload of arbitrary size with the standard recipe."""
-    return _contig(name, seed, B, N, H, D, k_offset=k_offset, rope=rope)
+def custom(seed, B, N, H, D, *, k_offset=True, rope=True, Hkv=None, Nkv=None,
+           name="custom") -> Workload:
+    """A contiguous workload of arbitrary size with the standard recipe
+    (GQA when ``Hkv`` < ``H``; cross-length when ``Nkv`` != ``N``, which
+    the RoPE/RMSNorm preparation does not accept)."""
+    return _contig(name, seed, B, N, H, D, k_offset=k_offset, rope=rope, Hkv=Hkv, Nkv=Nkv)

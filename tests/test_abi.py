@@ -1,0 +1,119 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+that include/qattn.h declares, and refuses invalid arguments by name before
+touching the GPU (so these run without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_exact_attention_qattn_b200 as qa
+from quantized_exact_attention_qattn_b200 import _lib
+from quantized_exact_attention_qattn_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return qa.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qattn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    assert set(names) == set(_lib.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.qattn_version().decode().startswith("qattn-b200")
+
+
+def _view(ptr=0x1000, strides=(1 << 20, 512, 128, 1)):
+    v = _lib.BNHD()
+    v.ptr = ptr
+    for i, s in enumerate(strides):
+        v.stride[i] = s
+    return v
+
+
+FAKE = 0x7f0000001000        # never dereferenced: every call below is refused first
+
+
+def test_fwd_refusals(lib):
+    args = dict(B=1, Nq=128, Nkv=128, Hq=2, Hkv=2, D=128)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.qattn_fwd(a["B"], a["Nq"], a["Nkv"], a["Hq"], a["Hkv"], a["D"], kw.get("q8", FAKE),
+                             FAKE, FAKE, FAKE, kw.get("mode", 0), FAKE, FAKE,
+                             kw.get("sm_scale", 0.0), kw.get("out", FAKE), kw.get("err", FAKE), None)
+    assert call(D=96) == 4
+    assert call(Hq=3) == 4
+    assert call(Nq=0) == 2
+    assert call(B=-1) == 2
+    assert call(mode=2) == 4
+    assert call(sm_scale=-1.0) == 4
+    assert call(sm_scale=float("nan")) == 4
+    assert call(q8=None) == 1
+    assert call(err=None) == 1
+    assert call(out=FAKE + 2) == 3
+    assert "16-byte" in lib.qattn_last_error().decode()
+
+
+def test_prep_refusals(lib):
+    def call(rot=96, q=None, D=128, eps=1e-5, theta=10000.0):
+        return lib.qattn_prep(1, 8, 2, 2, D, q or _view(), _view(), FAKE, FAKE, eps, rot, theta, 0,
+                              FAKE, FAKE, None)
+    assert call(rot=95) == 4
+    assert call(rot=8) == 4              # not a multiple of 16
+    assert call(rot=144) == 4            # larger than D
+    assert call(theta=0.0) == 4
+    assert call(eps=-1.0) == 4
+    assert call(D=100) == 4
+    assert call(q=_view(strides=(1 << 20, 512, 128, 2))) == 3
+    assert call(q=_view(strides=(1 << 20, 516, 128, 1))) == 3
+    assert call(q=_view(ptr=FAKE + 8)) == 3
+    assert call(q=_view(ptr=0)) == 1
+
+
+def test_quant_refusals_and_workspace_query(lib):
+    need = lib.qattn_quant_workspace_bytes(1, 37810, 56, 128)
+    nk = (37810 + 63) // 64
+    assert need >= nk * 56 * 128 * (8 + 4) + 56 * 128 * 4
+    assert lib.qattn_quant_workspace_bytes(1, 0, 56, 128) == 0
+    assert lib.qattn_quant_workspace_bytes(1, 10, 56, 96) == 0
+
+    def call(ws=FAKE, nbytes=None, v=None, k_mean=FAKE):
+        return lib.qattn_quant(1, 37810, 37810, 56, 56, 128, _view(), _view(), v or _view(),
+                               FAKE, FAKE, FAKE, FAKE, k_mean, FAKE, FAKE, ws,
+                               need if nbytes is None else nbytes, None)
+    assert call(nbytes=need - 1) == 5
+    assert call(ws=None) == 5
+    assert call(k_mean=None) == 1
+    assert call(v=_view(strides=(1 << 20, 512, 100, 1))) == 3
+    assert "workspace" in (lib.qattn_quant(1, 64, 64, 1, 1, 128, _view(), _view(), _view(), FAKE,
+                                           FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) and
+                           lib.qattn_last_error().decode())
+
+
+def test_hadamard_needs_power_of_four_head_dim(lib):
+    need = lib.qattn_quant_workspace_bytes(1, 64, 1, 128)
+    st = lib.qattn_quant_hadamard(1, 64, 64, 1, 1, 128, _view(), _view(), _view(), FAKE, FAKE,
+                                  FAKE, FAKE, FAKE, FAKE, FAKE, need, None)
+    assert st == 4 and "Hadamard" in lib.qattn_last_error().decode()
+
+
+def test_scores_refusals(lib):
+    assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) == 2
+    assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, None, 4, FAKE, FAKE, None) == 1
+    assert lib.qattn_check(None, None) == 1

@@ -1,0 +1,160 @@
+"""Edge shapes, GQA, cross-length, metamorphic and sentinel checks on the GPU.
+
+Ragged sequence lengths exercise partial 32-row Q groups, partial 128-row Q
+tiles, partial 64-key tiles (masked scores, zero V rows) and single-row cases;
+the p2 validation grid (1/2/6/7 rows, 1..768 keys) appears through N.
+"""
+import numpy as np
+import pytest
+import torch
+
+import quantized_exact_attention_qattn_b200 as qa
+from quantized_exact_attention_qattn_b200 import synth
+from oracle import qattn_oracle as O
+
+from gpu_helpers import DEV, assert_out_close, dev_bf16, host, oracle_full, run_pipeline
+
+pytestmark = pytest.mark.gpu
+
+EDGE = [
+    # (B, N, H, Hkv, D, rope)
+    (1, 1, 1, 1, 128, True),
+    (1, 2, 2, 2, 64, False),
+    (1, 7, 1, 1, 256, True),
+    (2, 15, 2, 1, 128, True),
+    (1, 17, 3, 3, 64, False),
+    (1, 31, 2, 2, 256, False),
+    (1, 64, 2, 2, 128, True),
+    (1, 65, 4, 2, 128, True),
+    (3, 129, 2, 2, 64, False),
+    (1, 200, 8, 2, 256, True),
+    (1, 729, 2, 2, 64, False),
+    (2, 768, 2, 2, 128, True),
+    (1, 1000, 6, 3, 128, True),
+]
+
+
+def _check_all(w, pipe, ref):
+    for key in ("qp", "kp", "k_mean", "q8", "q_scale", "k8", "k_scale", "v8t", "v_scale"):
+        assert np.array_equal(host(getattr(pipe, key)), ref[key]), key
+    assert_out_close(host(pipe.out), ref["out"], w.name)
+
+
+@pytest.mark.parametrize("B,N,H,Hkv,D,rope", EDGE)
+def test_edge_shapes(B, N, H, Hkv, D, rope):
+    w = synth.custom(1000 + N, B, N, H, D, rope=rope, Hkv=Hkv)
+    pipe = run_pipeline(w)
+    _check_all(w, pipe, oracle_full(w))
+
+
+@pytest.mark.parametrize("Nq,Nkv,Hq,Hkv,D", [(100, 300, 4, 2, 128), (300, 65, 2, 1, 64),
+                                             (1, 129, 2, 2, 256)])
+def test_cross_length_without_prep(Nq, Nkv, Hq, Hkv, D):
+    w = synth.custom(7 + Nq, 1, Nq, Hq, D, Hkv=Hkv, Nkv=Nkv, rope=False)
+    pipe = qa.Pipeline(1, Nq, Nkv, Hq, Hkv, D, prep=False, device=DEV)
+    pipe.run(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v))
+    pipe.check()
+    q8, qs = O.quant_q(w.q)
+    k8, ks = O.quant_k(w.k, O.k_mean(w.k))
+    v8t, vs = O.quant_v(w.v)
+    out, _, _ = O.attention(q8, qs, k8, ks, v8t, vs, Nkv)
+    assert np.array_equal(host(pipe.q8), q8) and np.array_equal(host(pipe.k8), k8)
+    assert np.array_equal(host(pipe.v8t), v8t)
+    assert_out_close(host(pipe.out), out, "cross-length")
+
+
+@pytest.mark.parametrize("Nq,Nkv,Hq,Hkv,D", [(65, 200, 4, 1, 256), (130, 97, 2, 2, 64),
+                                             (1, 64, 8, 4, 256)])
+def test_hadamard_small(Nq, Nkv, Hq, Hkv, D):
+    w = synth.make("gqa_chunk", Nq=Nq, Nkv=Nkv, Hq=Hq, Hkv=Hkv, D=D, seed=Nq + Nkv)
+    pipe = run_pipeline(w)
+    ref = oracle_full(w)
+    for key in ("q8", "q_scale", "k8", "k_scale", "v8t", "v_scale"):
+        assert np.array_equal(host(getattr(pipe, key)), ref[key]), key
+    assert_out_close(host(pipe.out), ref["out"], "hadamard")
+
+
+def test_interleaved_strided_equals_contiguous():
+    # GPU-vs-GPU: the interleaved QKV buffer and contiguous copies give identical bytes
+    B, N, H, D = 1, 333, 4, 128
+    rng = np.random.default_rng(5)
+    buf = torch.from_numpy(rng.standard_normal((B, N, 3, H, D), dtype=np.float32)).to(torch.bfloat16).to(DEV)
+    w = synth.custom(5, B, N, H, D)
+    qw, kw = dev_bf16(w.q_weight), dev_bf16(w.k_weight)
+    a = qa.Pipeline(B, N, N, H, H, D, device=DEV)
+    a.run(buf[:, :, 0], buf[:, :, 1], buf[:, :, 2], qw, kw, 1e-5, 96)
+    b = qa.Pipeline(B, N, N, H, H, D, device=DEV)
+    b.run(buf[:, :, 0].contiguous(), buf[:, :, 1].contiguous(), buf[:, :, 2].contiguous(), qw, kw,
+          1e-5, 96)
+    a.check(); b.check()
+    assert torch.equal(a.out.view(torch.int16), b.out.view(torch.int16))
+    assert torch.equal(a.v8t, b.v8t)
+
+
+def test_batch_entries_are_independent():
+    w = synth.custom(6, 3, 150, 2, 64, rope=False)
+    full = run_pipeline(w)
+    for bi in range(3):
+        one = synth.custom(6, 3, 150, 2, 64, rope=False)
+        one.q, one.k, one.v, one.B = one.q[bi:bi + 1], one.k[bi:bi + 1], one.v[bi:bi + 1], 1
+        p1 = run_pipeline(one)
+        assert torch.equal(p1.out.view(torch.int16), full.out[bi:bi + 1].view(torch.int16))
+
+
+def test_head_permutation_permutes_output():
+    w = synth.custom(8, 1, 200, 4, 128)
+    base = run_pipeline(w)
+    perm = [2, 0, 3, 1]
+    w2 = synth.custom(8, 1, 200, 4, 128)
+    w2.q, w2.k, w2.v = w.q[:, :, perm], w.k[:, :, perm], w.v[:, :, perm]
+    p2 = run_pipeline(w2)
+    assert torch.equal(p2.out.view(torch.int16), base.out[:, :, perm].view(torch.int16))
+
+
+def test_outputs_leave_neighbouring_memory_untouched():
+    # each output is a window inside a larger buffer of sentinel bytes
+    B, N, H, D = 1, 77, 2, 128
+    w = synth.custom(9, B, N, H, D)
+    q, k, v = dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.v)
+    pad = 4096
+
+    def window(shape, dtype, fill):
+        n = int(np.prod(shape))
+        big = torch.full((n + 2 * pad,), fill, dtype=dtype, device=DEV)
+        return big, big[pad:pad + n].view(shape)
+
+    qp_b, qp = window((B, N, H, D), torch.int16, -12345)
+    kp_b, kp = window((B, N, H, D), torch.int16, -12345)
+    qattn_args = (B, N, H, H, D)
+    qa.qattn_prep(*qattn_args, q, k, dev_bf16(w.q_weight), dev_bf16(w.k_weight), 1e-5, 96, 1e4, 0,
+                  qp, kp)
+    nk = O.ceil_div(N, 64)
+    q8_b, q8 = window((B, H, N, D), torch.int8, 77)
+    k8_b, k8 = window((B, H, N, D), torch.int8, 77)
+    qs_b, qs = window((B, H, 4 * O.ceil_div(N, 128)), torch.float32, 123.0)
+    ks_b, ks = window((B, H, nk), torch.float32, 123.0)
+    mu_b, mu = window((B, H, D), torch.float32, 123.0)
+    v8_b, v8 = window((B, H, D, 64 * nk), torch.uint8, 0xAB)
+    vs_b, vs = window((B, H, D), torch.float32, 123.0)
+    ws = torch.empty(qa.qattn_quant_workspace_bytes(B, N, H, D), dtype=torch.uint8, device=DEV)
+    qa.qattn_quant(B, N, N, H, H, D, qp.view(torch.bfloat16), kp.view(torch.bfloat16), v, q8, qs,
+                   k8, ks, mu, v8, vs, ws)
+    out_b, out = window((B, N, H, D), torch.int16, 0x5A5A)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    qa.qattn_fwd(B, N, N, H, H, D, q8, qs, k8, ks, 0, v8, vs, 0.0, out, err)
+    qa.qattn_check(err)
+    for big, fill in ((qp_b, -12345), (kp_b, -12345), (q8_b, 77), (k8_b, 77), (qs_b, 123.0),
+                      (ks_b, 123.0), (mu_b, 123.0), (v8_b, 0xAB), (vs_b, 123.0), (out_b, 0x5A5A)):
+        assert bool((big[:pad] == fill).all()) and bool((big[-pad:] == fill).all())
+    ref = oracle_full(w)
+    assert_out_close(host(out.view(torch.bfloat16)), ref["out"], "windowed")
+    assert np.array_equal(host(v8), ref["v8t"])       # padded key rows are written as 0x00
+
+
+def test_repeat_calls_are_deterministic():
+    w = synth.make("mid")
+    a = run_pipeline(w)
+    first = a.out.clone()
+    a.run_fwd()
+    a.check()
+    assert torch.equal(first.view(torch.int16), a.out.view(torch.int16))

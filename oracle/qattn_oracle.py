@@ -328,12 +328,18 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
 
     per query row:  m = -5e6f, d = 1.0f, RO = 0
     for each 64-key tile t = 0, 1, ... in increasing order:
-      s_j   = ((f32)S_j * (q_s * k_s)) * c      (FP32; c = log2(e)/sqrt(D);
-                                                 keys past N get -5e6f)
+      A     = (q_s * k_s) * c                   (FP32 dequantization x softmax
+                                                 scale, c = log2(e)/sqrt(D))
+      s_j   = (f32)S_j * A                      (scaled score, FP32; keys past N
+                                                 get -5e6f)
       mt    = max_j s_j - 8.807f
       mn    = max(m, mt)
       old   = 2^(m - mn);  d *= old;  RO *= old
-      p_j   = 2^(s_j - mn)                      (FP32 value of exp2 in FP64)
+      p_j   = 2^fma(S_j, A, -mn)                (reading of "the reference fused
+                                                 multiply-add placement": the
+                                                 exponent is S*A - mn rounded
+                                                 once; 2^x is the FP32 value of
+                                                 exp2 in FP64; masked keys: 0)
       d    += p_j, j ascending, FP32, unquantized p
       P8_j  = e4m3_rn_satfinite(p_j)
       RO   += sum_j P8_j * V8[j, :]             (reading: exact tile sum, FP64)
@@ -365,23 +371,29 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
         j0, j1 = t * KV_TILE, min(n_kv, (t + 1) * KV_TILE)
         kt = k8[:, kvh, j0:j1].astype(np.float64)                    # [B,Hq,w,D]
         s_int = np.matmul(qsel, np.swapaxes(kt, -1, -2))             # exact integers
-        sf = s_int.astype(F32)
+        sf = s_int.astype(F32)                                       # exact (|S| < 2^24)
         if k_scale_mode == 0:
             ks = k_scale[:, kvh, t].astype(F32)                      # [B,Hq]
-            alpha = (qs * ks[:, :, None]).astype(F32)[..., None]     # [B,Hq,R,1]
+            a = ((qs * ks[:, :, None]).astype(F32) * c).astype(F32)[..., None]   # [B,Hq,R,1]
         else:
             ks = f32_from_f16_bits(k_scale[:, kvh, j0:j1])           # [B,Hq,w]
-            alpha = (qs[..., None] * ks[:, :, None, :]).astype(F32)  # [B,Hq,R,w]
-        s = ((sf * alpha).astype(F32) * c).astype(F32)
-        if j1 - j0 < KV_TILE:                                        # masked tail
-            pad = np.full(s.shape[:-1] + (KV_TILE - (j1 - j0),), MASKED_SCORE, F32)
+            a = ((qs[..., None] * ks[:, :, None, :]).astype(F32) * c).astype(F32)  # [B,Hq,R,w]
+        s = (sf * a).astype(F32)
+        w = j1 - j0
+        if w < KV_TILE:                                              # masked tail
+            pad = np.full(s.shape[:-1] + (KV_TILE - w,), MASKED_SCORE, F32)
             s = np.concatenate([s, pad], axis=-1)
         mt = (np.max(s, axis=-1) - FP8_OFFSET).astype(F32)
         mn = np.maximum(m, mt)
         old = np.exp2((m - mn).astype(F32).astype(np.float64)).astype(F32)
         den = (den * old).astype(F32)
         ro = ro * old.astype(np.float64)[..., None]
-        p = np.exp2((s - mn[..., None]).astype(F32).astype(np.float64)).astype(F32)
+        # fma(S, A, -mn): the float64 product S*A is exact (22 + 24 bits) and the
+        # float64 difference is exact or below half a float32 ulp of rounding
+        e = (s_int * a.astype(np.float64) - mn.astype(np.float64)[..., None]).astype(F32)
+        p = np.exp2(e.astype(np.float64)).astype(F32)
+        if w < KV_TILE:
+            p = np.concatenate([p, np.zeros(p.shape[:-1] + (KV_TILE - w,), F32)], axis=-1)
         for j in range(KV_TILE):
             den = (den + p[..., j]).astype(F32)
         p8 = e4m3_value_from_f32(p)[..., : j1 - j0]                   # exact values

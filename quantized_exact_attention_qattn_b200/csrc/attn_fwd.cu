@@ -44,8 +44,8 @@ constexpr float kMasked = -5000000.0f;
 template <int D, int NQT>
 struct Cfg {
   static constexpr int STAGES = (D == 256) ? 3 : 4;
-  static constexpr int KCH = (D >= 128) ? 128 : 64;       // K-major swizzle row width (bytes)
-  static constexpr int NCH = D / KCH;                      // 128-byte column chunks per row
+  static constexpr int KCH = (D >= 128) ? 128 : 64;        // K-major swizzle row width (bytes)
+  static constexpr int NCH = D / KCH;                       // column chunks per row
   static constexpr uint32_t SW_QK = (KCH == 128) ? 2u : 4u; // 128B or 64B swizzle
   static constexpr int Q_BYTES = BM * D;
   static constexpr int K_BYTES = BN * D;
@@ -53,15 +53,22 @@ struct Cfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = SMEM_Q + NQT * Q_BYTES;
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
-  static constexpr int SMEM_BAR = SMEM_V + STAGES * V_BYTES;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NQT + 1;
+  static constexpr int SMEM_OLD = SMEM_V + STAGES * V_BYTES;        // float [NQT][2][128]
+  static constexpr int SMEM_DEN = SMEM_OLD + NQT * 2 * BM * 4;      // float [NQT][128]
+  static constexpr int SMEM_BAR = SMEM_DEN + NQT * BM * 4;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 11 * NQT;
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
-  static constexpr int THREADS = 128 + 128 * NQT;
+  // warps 0-3: producer, one MMA issuer per query tile, spare; then NQT softmax
+  // warpgroups; then the correction warpgroup
+  static constexpr int SOFTMAX_WARP0 = 4;
+  static constexpr int CORR_WARP0 = 4 + 4 * NQT;
+  static constexpr int THREADS = 32 * (CORR_WARP0 + 4);
+  // tensor memory columns: O[NQT] (D each), S[NQT] (64 each), P[NQT][2] (16 each)
   static constexpr uint32_t O_COL = 0;
   static constexpr uint32_t S_COL = NQT * D;
   static constexpr uint32_t P_COL = S_COL + NQT * BN;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(P_COL + NQT * (BN / 4) <= TMEM_COLS, "tensor memory budget");
+  static_assert(P_COL + NQT * 2 * (BN / 4) <= TMEM_COLS, "tensor memory budget");
   static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
   static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
 };
@@ -72,11 +79,76 @@ struct FwdParams {
   const float* v_scale;
   uint16_t* out;
   int* dev_err;
-  int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups, k_scale_mode;
+  int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups;
   float c;
 };
 
-template <int D, int NQT>
+// ---------------------------------------------------------------- exp2
+// Columns j with (j % 8) < kPolyPer8 evaluate 2^t with an FMA-pipe polynomial,
+// the rest with the MUFU ex2.approx, so both pipes share the exponentials.
+#ifndef QATTN_POLY_PER8
+#define QATTN_POLY_PER8 0
+#endif
+constexpr int kPolyPer8 = QATTN_POLY_PER8;
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: x + kMagic rounds x to an integer
+// 2^f on [-1/2, 1/2], degree 5, relative minimax (fit_exp2.py), max relative error
+// 2.3e-7 in FP32: about that of ex2.approx, so both paths round P to E4M3 alike.
+constexpr float kC0 = 1.000000119e+00f, kC1 = 6.931469440e-01f, kC2 = 2.402212024e-01f,
+                kC3 = 5.550713092e-02f, kC4 = 9.675540961e-03f, kC5 = 1.327647245e-03f;
+
+// 2^t for two values at once: n = round(t), f = t - n, 2^t = poly(f) * 2^n with
+// n added to the exponent field.  t is clamped at -126 so that the exponent of
+// the result stays >= 0 (a tiny or subnormal positive value, never a wrap).
+__device__ __forceinline__ float2 exp2_poly2(float2 t) {
+  t.x = fmaxf(t.x, -126.0f);
+  t.y = fmaxf(t.y, -126.0f);
+  const float2 j = fadd2(t, make_float2(kMagic, kMagic));          // round to integer
+  const float2 n = fadd2(j, make_float2(-kMagic, -kMagic));        // exact
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), t);         // t - n, exact
+  float2 q = ffma2(make_float2(kC5, kC5), f, make_float2(kC4, kC4));
+  q = ffma2(q, f, make_float2(kC3, kC3));
+  q = ffma2(q, f, make_float2(kC2, kC2));
+  q = ffma2(q, f, make_float2(kC1, kC1));
+  q = ffma2(q, f, make_float2(kC0, kC0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
+}
+
+template <int J>
+__device__ __forceinline__ float2 exp2_pair(float2 t) {
+  if constexpr ((J % 8) < kPolyPer8) {
+    return exp2_poly2(t);
+  } else {
+    return make_float2(ex2_approx(t.x), ex2_approx(t.y));
+  }
+}
+
+// x[j] holds the exact FP32 score S_j; the exponent is fma(S_j, A, -mn).
+template <int J>
+__device__ __forceinline__ void exp_block(float (&x)[64], float2 a2, float2 nb2) {
+  if constexpr (J < 64) {
+    const float2 t = ffma2(make_float2(x[J], x[J + 1]), a2, nb2);
+    const float2 e = exp2_pair<J>(t);
+    x[J] = e.x;
+    x[J + 1] = e.y;
+    exp_block<J + 2>(x, a2, nb2);
+  }
+}
+
+template <int J>
+__device__ __forceinline__ void exp_block_masked(float (&x)[64], float2 a2, float2 nb2, int nvalid) {
+  if constexpr (J < 64) {
+    float2 t = ffma2(make_float2(x[J], x[J + 1]), a2, nb2);
+    if (J >= nvalid) t.x = -INFINITY;
+    if (J + 1 >= nvalid) t.y = -INFINITY;
+    const float2 e = exp2_pair<J>(t);
+    x[J] = e.x;
+    x[J + 1] = e.y;
+    exp_block_masked<J + 2>(x, a2, nb2, nvalid);
+  }
+}
+
+template <int D, int NQT, int KMODE>
 __global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -84,21 +156,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  float* old_s = reinterpret_cast<float*>(smem + C::SMEM_OLD);     // [NQT][2][BM]
+  float* den_s = reinterpret_cast<float*>(smem + C::SMEM_DEN);     // [NQT][BM]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_full = q_full + 1;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;
-  uint64_t* p_full = s_full + NQT;
-  uint64_t* o_done = p_full + NQT;
-  uint64_t* drain = o_done + NQT;
+  // A parity wait for phase k is only sound if phase k+1 cannot complete before
+  // the waiter is through.  Where the producer side could run two phases ahead
+  // (rescale factors, P buffers and the P.V products that read them) there is
+  // one barrier per buffer, indexed [i][t & 1]; every other barrier's next phase
+  // depends on its waiter having passed (checked per barrier below).
+  uint64_t* s_full = kv_empty + C::STAGES;   // MMA -> softmax: S_i(t) in TMEM
+  uint64_t* s_free = s_full + NQT;           // softmax -> MMA: S_i(t) read
+  uint64_t* o_rdy = s_free + NQT;            // correction -> MMA: O_i rescaled for t
+  uint64_t* fin = o_rdy + NQT;               // softmax -> correction: final denominators
+  uint64_t* old_rdy = fin + NQT;             // [NQT][2] softmax -> correction: old(t) in smem
+  uint64_t* p_full = old_rdy + 2 * NQT;      // [NQT][2] softmax -> MMA: P_i(t) in TMEM
+  uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax/correction: PV_i(t) done
+  uint64_t* drain = pv_done + 2 * NQT;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (b, h, group of NQT query tiles), tiles of one head adjacent
   const int item = blockIdx.x;
   const int grp = item % p.n_groups;
   const int bh = item / p.n_groups;
@@ -115,14 +197,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(q_full, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(kv_empty + s, nvalid);      // one commit per MMA issuer
     }
     for (int i = 0; i < NQT; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 4);
-      mbar_init(o_done + i, 1);
+      // arrivals from softmax / correction warpgroups: one elected lane per warp
+      mbar_init(s_free + i, 4);
+      mbar_init(o_rdy + i, 4);
+      mbar_init(fin + i, 4);
+      for (int bb = 0; bb < 2; ++bb) {
+        mbar_init(old_rdy + 2 * i + bb, 4);
+        mbar_init(p_full + 2 * i + bb, 4);
+        mbar_init(pv_done + 2 * i + bb, 1);
+      }
     }
-    mbar_init(drain, 1);
+    for (int i = 0; i < NQT; ++i) mbar_init(drain + i, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -159,194 +248,280 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN, 0, bhkv);
         issued = t + 1;
       }
-      // drain: every issued copy must land before the CTA may exit
-      int dummy = 0;
+      int dummy = 0;      // drain: every issued copy must land before the CTA may exit
       mbar_wait(q_full, 0, &dummy, p.dev_err, kErrTimeoutDrain);
       for (int u = max(0, issued - C::STAGES); u < issued; ++u)
         mbar_wait(kv_full + (u % C::STAGES), (u / C::STAGES) & 1, &dummy, p.dev_err,
                   kErrTimeoutDrain);
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+  } else if (warp <= NQT) {
+    // ================================================================ MMA issuers
+    // One issuing thread per query tile i (warp 1 + i), so the two tiles' chains
+    // never wait on each other: QK_i(t+1) as soon as S_i(t) has been read, then
+    // PV_i(t) once P_i(t) is written and O_i rescaled.
+    const int i = warp - 1;
+    if (lane == 0 && i < nvalid) {
+      const uint32_t sQ = smem_u32(smem + C::SMEM_Q) + i * C::Q_BYTES;
       const uint32_t sK = smem_u32(smem + C::SMEM_K);
       const uint32_t sV = smem_u32(smem + C::SMEM_V);
-      auto issue_qk = [&](int i, int s) {
-        const uint32_t d_tm = tmem + C::S_COL + i * BN;
+      const uint32_t tS = tmem + C::S_COL + i * BN;
+      const uint32_t tO = tmem + C::O_COL + i * D;
+      auto issue_qk = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
-          const uint64_t ad = smem_desc(sQ + i * C::Q_BYTES + ch * (BM * C::KCH) + off,
-                                        8 * C::KCH, C::SW_QK);
+          const uint64_t ad = smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          mma_i8_ss(d_tm, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_i8_ss(tS, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         tc_commit(s_full + i);
       };
-      auto issue_pv = [&](int i, int s, int t) {
-        const uint32_t d_tm = tmem + C::O_COL + i * D;
-        const uint32_t a_tm = tmem + C::P_COL + i * (BN / 4);
+      auto issue_pv = [&](int s, int t) {
+        const uint32_t a_tm = tmem + C::P_COL + (i * 2 + (t & 1)) * (BN / 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 32; ++kk) {
           const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
-          mma_f8_ts(d_tm, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(o_done + i);
+        tc_commit(pv_done + 2 * i + (t & 1));
       };
       bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ);
       if (ok) ok = mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV);
       if (ok) {
         tc_fence_after();
-        for (int i = 0; i < nvalid; ++i) issue_qk(i, 0);
+        issue_qk(0);
       }
       for (int t = 0; ok && t < nK; ++t) {
         const int s = t % C::STAGES;
-        const int s1 = (t + 1) % C::STAGES;
-        bool next_ready = false;
-        for (int i = 0; ok && i < nvalid; ++i) {
-          ok = mbar_wait(p_full + i, t & 1, abort, p.dev_err, kErrTimeoutP);
+        if (t + 1 < nK) {
+          const int s1 = (t + 1) % C::STAGES;
+          ok = mbar_wait(kv_full + s1, ((t + 1) / C::STAGES) & 1, abort, p.dev_err, kErrTimeoutKV) &&
+               mbar_wait(s_free + i, t & 1, abort, p.dev_err, kErrTimeoutS);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(i, s, t);
-          if (t + 1 < nK) {
-            if (!next_ready) {
-              ok = mbar_wait(kv_full + s1, ((t + 1) / C::STAGES) & 1, abort, p.dev_err,
-                             kErrTimeoutKV);
-              if (!ok) break;
-              tc_fence_after();
-              next_ready = true;
-            }
-            issue_qk(i, s1);
-          }
+          issue_qk(s1);
         }
-        if (ok) tc_commit(kv_empty + s);
+        ok = mbar_wait(p_full + 2 * i + (t & 1), (t >> 1) & 1, abort, p.dev_err, kErrTimeoutP) &&
+             mbar_wait(o_rdy + i, t & 1, abort, p.dev_err, kErrTimeoutO);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(s, t);
+        tc_commit(kv_empty + s);   // stage s is free once every issuer's reads finished
       }
-      // drain: wait for every issued tensor-core operation before tear-down
-      tc_commit(drain);
+      tc_commit(drain + i);        // drain: every issued tensor-core op before tear-down
       int dummy = 0;
-      mbar_wait(drain, 0, &dummy, p.dev_err, kErrTimeoutDrain);
+      mbar_wait(drain + i, 0, &dummy, p.dev_err, kErrTimeoutDrain);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= C::SOFTMAX_WARP0 && warp < C::CORR_WARP0) {
     // ================================================================ softmax
-    const int wg = (warp - 4) >> 2;
+    const int wg = (warp - C::SOFTMAX_WARP0) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     if (wg < nvalid) {
       const int qt = qt0 + wg;
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
       const uint32_t tS = tmem + lane_off + C::S_COL + wg * BN;
-      const uint32_t tP = tmem + lane_off + C::P_COL + wg * (BN / 4);
-      const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
+      const uint32_t tP = tmem + lane_off + C::P_COL + (wg * 2) * (BN / 4);
       const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
       const int last_valid = p.Nkv - (nK - 1) * BN;
+      const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
+      const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
       float m = kMInit, den = 1.0f;
+      float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
       bool ok = true;
       for (int t = 0; t < nK; ++t) {
-        // warp-uniform outcome: the tcgen05.ld / shuffles below are warp-collective
+        float ks_cur = ks_next;
+        if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sraw[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+        float x[64];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
         tmem_wait_ld();
-        float sv[64];
-        if (p.k_scale_mode == 0) {
-          const float ks = static_cast<const float*>(p.k_scale)[static_cast<int64_t>(bhkv) * nK + t];
-          const float alpha = __fmul_rn(qs, ks);
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            sv[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(sraw[j])), alpha), p.c);
-        } else {
-          const __half* ks16 = static_cast<const __half*>(p.k_scale) +
-                               static_cast<int64_t>(bhkv) * p.Nkv + t * BN;
-          const int nv = (t == nK - 1) ? last_valid : BN;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float ks = (j < nv) ? __half2float(ks16[j]) : 0.0f;
-            sv[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(sraw[j])),
-                                        __fmul_rn(qs, ks)), p.c);
-          }
-        }
-        if (t == nK - 1) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j >= last_valid) sv[j] = kMasked;
-        }
-        float mx = sv[0];
-#pragma unroll
-        for (int j = 1; j < 64; ++j) mx = fmaxf(mx, sv[j]);
-        const float mn = fmaxf(m, __fsub_rn(mx, kFp8Offset));
-        const float old = ex2_approx(__fsub_rn(m, mn));
-        den = __fmul_rn(den, old);
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 64; j += 4) {
-          const float p0 = ex2_approx(__fsub_rn(sv[j], mn));
-          const float p1 = ex2_approx(__fsub_rn(sv[j + 1], mn));
-          const float p2 = ex2_approx(__fsub_rn(sv[j + 2], mn));
-          const float p3 = ex2_approx(__fsub_rn(sv[j + 3], mn));
-          den = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(den, p0), p1), p2), p3);
-          pk[j / 4] = static_cast<uint32_t>(cvt_e4m3x2(p0, p1)) |
-                      (static_cast<uint32_t>(cvt_e4m3x2(p2, p3)) << 16);
-        }
-        if (t > 0) {
-          // PV(t-1) must be finished: it reads P and accumulates into O
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(o_done + wg, (t - 1) & 1, abort, p.dev_err, kErrTimeoutO));
-          if (!ok) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, old != 1.0f)) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(tO + c0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__fmul_rn(__uint_as_float(o[j]), old));
-              tmem_st32(tO + c0, o);
-            }
-          }
-        }
-        tmem_st16(tP, pk);
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + wg);
+        if (lane == 0) mbar_arrive(s_free + wg);
+        // INT32 score -> FP32 (exact for |S| < 2^22): the bits of kMagic + S, then
+        // minus kMagic (exact)
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(__float_as_uint(x[j]) + 0x4B400000u);
+        const bool last = (t == nK - 1);
+        float mn;
+        float2 a2, nb2;
+        if constexpr (KMODE == 0) {
+          // A = (q_scale * k_scale) * c; tile max of S*A from the max of S (A > 0)
+          if (last) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (j >= last_valid) x[j] = 0.0f;          // below every valid kMagic + S
+          }
+          float mq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            mq[q] = x[16 * q];
+#pragma unroll
+            for (int j = 1; j < 16; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
+          }
+          const float xmax = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+            x[j] = sj.x;
+            x[j + 1] = sj.y;
+          }
+          const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
+          const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+          mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
+          a2 = make_float2(a, a);
+          nb2 = make_float2(-mn, -mn);
+        } else {
+          // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent uses
+          // fma(S_j, A_j, -mn), so x[] keeps S_j and a[] keeps A_j
+          // (A_j is recomputed in the second pass instead of held in registers)
+          const int nv = last ? last_valid : BN;
+          float smx = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float ksj = (j < nv) ? __half2float(ks16[t * BN + j]) : 0.0f;
+            x[j] = __fsub_rn(x[j], kMagic);
+            if (j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c)));
+          }
+          mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float ksj = (j < nv) ? __half2float(ks16[t * BN + j]) : 0.0f;
+            x[j] = __fmaf_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c), -mn);
+          }
+          a2 = make_float2(1.0f, 1.0f);
+          nb2 = make_float2(0.0f, 0.0f);
+        }
+        const float old = ex2_approx(__fsub_rn(m, mn));
+        old_s[(wg * 2 + (t & 1)) * BM + row] = old;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(old_rdy + 2 * wg + (t & 1));
+        if (last) {
+          exp_block_masked<0>(x, a2, nb2, last_valid);
+        } else {
+          exp_block<0>(x, a2, nb2);
+        }
+        // denominator: unquantized probabilities, four independent pair sums
+        float2 acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
+#pragma unroll
+        for (int j = 8; j < 64; j += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
+        }
+        acc[0] = fadd2(acc[0], acc[1]);
+        acc[2] = fadd2(acc[2], acc[3]);
+        acc[0] = fadd2(acc[0], acc[2]);
+        den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 64; j += 4)
+          pk[j / 4] = static_cast<uint32_t>(cvt_e4m3x2(x[j], x[j + 1])) |
+                      (static_cast<uint32_t>(cvt_e4m3x2(x[j + 2], x[j + 3])) << 16);
+        if (t >= 2) {   // P buffer (t & 1) was read by PV_i(t-2)
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + (t & 1), ((t >> 1) - 1) & 1,
+                                                 abort, p.dev_err, kErrTimeoutO));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        tmem_st16(tP + (t & 1) * (BN / 4), pk);
+        tmem_wait_st();
+        tc_fence_before();
+        if (last) den_s[wg * BM + row] = den;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(p_full + 2 * wg + (t & 1));
+          if (last) mbar_arrive(fin + wg);
+        }
         m = mn;
       }
-      // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + wg, (nK - 1) & 1, abort, p.dev_err,
-                                                    kErrTimeoutO));
-      if (ok) {
-        tc_fence_after();
-        const float inv = rcp_approx(den);
-        const int n = qt * BM + row;
-        const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
-        uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
+      (void)ok;
+    }
+  } else if (warp >= C::CORR_WARP0) {
+    // ================================================================ correction
+    // Rescales O_i by old(t) between PV_i(t-1) and PV_i(t) (only warps in which
+    // some row's maximum moved), then normalises and stores the output.
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    bool ok = true;
+    for (int t = 0; ok && t < nK; ++t) {
+      for (int i = 0; i < nvalid; ++i) {
+        ok = __all_sync(0xffffffffu, mbar_wait(old_rdy + 2 * i + (t & 1), (t >> 1) & 1, abort,
+                                               p.dev_err, kErrTimeoutO));
+        if (!ok) break;
+        if (t > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
+                                                 abort, p.dev_err, kErrTimeoutO));
+          if (!ok) break;
+          tc_fence_after();
+          const float o = old_s[(i * 2 + (t & 1)) * BM + row];
+          if (__any_sync(0xffffffffu, o != 1.0f)) {
+            const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c0, o);
-          tmem_wait_ld();
-          if (n < p.Nq) {
-            uint32_t w[16];
+            for (int c0 = 0; c0 < D; c0 += 64) {
+              uint32_t r[64];
+              tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+              tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float a0 = __fmul_rn(__fmul_rn(__uint_as_float(o[j]), inv), vs[c0 + j]);
-              const float a1 = __fmul_rn(__fmul_rn(__uint_as_float(o[j + 1]), inv), vs[c0 + j + 1]);
-              w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a0))) |
-                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a1))) << 16);
+              for (int j = 0; j < 64; j += 2) {
+                const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                       make_float2(o, o));
+                r[j] = __float_as_uint(v.x);
+                r[j + 1] = __float_as_uint(v.y);
+              }
+              tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+              tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
             }
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-            d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            tmem_wait_st();
           }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_rdy + i);
+      }
+    }
+    // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only
+    for (int i = 0; ok && i < nvalid; ++i) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(pv_done + 2 * i + ((nK - 1) & 1), ((nK - 1) >> 1) & 1, abort,
+                                p.dev_err, kErrTimeoutO) &&
+                          mbar_wait(fin + i, 0, abort, p.dev_err, kErrTimeoutO));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = rcp_approx(den_s[i * BM + row]);
+      const int n = (qt0 + i) * BM + row;
+      const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
+      uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
+      const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c0, o);
+        tmem_wait_ld();
+        if (n < p.Nq) {
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                         make_float2(inv, inv)),
+                                   make_float2(vs[c0 + j], vs[c0 + j + 1]));
+            w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                       (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+          d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+          d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
         }
       }
     }
@@ -477,11 +652,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NQT>
+template <int D, int NQT, int KMODE>
 cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
                          const float* q_scale, const int8_t* k8, const void* k_scale,
-                         int k_scale_mode, const uint8_t* v8t, const float* v_scale, float c,
-                         uint16_t* out, int* dev_err, cudaStream_t st, const char** why) {
+                         const uint8_t* v8t, const float* v_scale, float c, uint16_t* out,
+                         int* dev_err, cudaStream_t st, const char** why) {
   using Cf = Cfg<D, NQT>;
   const int nQ = (Nq + BM - 1) / BM;
   const int nK = (Nkv + BN - 1) / BN;
@@ -499,15 +674,27 @@ cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* 
   p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale; p.out = out; p.dev_err = dev_err;
   p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
   p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
-  p.k_scale_mode = k_scale_mode; p.c = c;
+  p.c = c;
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) owns an SM
   const int smem = (Cf::SMEM_BYTES + 1024 > 116 * 1024) ? Cf::SMEM_BYTES + 1024 : 116 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT, KMODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(B) * Hq * p.n_groups);
-  attn_fwd_kernel<D, NQT><<<grid, Cf::THREADS, smem, st>>>(mQ, mK, mV, p);
+  attn_fwd_kernel<D, NQT, KMODE><<<grid, Cf::THREADS, smem, st>>>(mQ, mK, mV, p);
   return cudaGetLastError();
+}
+
+template <int D, int NQT>
+cudaError_t launch_fwd_d(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
+                         const float* q_scale, const int8_t* k8, const void* k_scale,
+                         int k_scale_mode, const uint8_t* v8t, const float* v_scale, float c,
+                         uint16_t* out, int* dev_err, cudaStream_t st, const char** why) {
+  if (k_scale_mode == 0)
+    return launch_fwd_t<D, NQT, 0>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, v8t, v_scale, c,
+                                   out, dev_err, st, why);
+  return launch_fwd_t<D, NQT, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, v8t, v_scale, c,
+                                 out, dev_err, st, why);
 }
 
 template <int D>
@@ -540,13 +727,13 @@ cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int
                        const char** why) {
   switch (D) {
     case 64:
-      return launch_fwd_t<64, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
+      return launch_fwd_d<64, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
                                  v_scale, score_c, out, dev_err, st, why);
     case 128:
-      return launch_fwd_t<128, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
+      return launch_fwd_d<128, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
                                   v8t, v_scale, score_c, out, dev_err, st, why);
     case 256:
-      return launch_fwd_t<256, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
+      return launch_fwd_d<256, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
                                   v8t, v_scale, score_c, out, dev_err, st, why);
     default:
       *why = "head dimension must be 64, 128 or 256";

@@ -490,3 +490,33 @@ def test_hadamard_reduces_kld_with_outlier_channels():
         ro.append(_kld_int8_k(kb, q, True, rng))
     assert np.mean(ro) < 0.3 * np.mean(un)
     assert np.mean(ro) < 1e-3
+
+
+def _f32_round_exact(fr):
+    """Correct float32 rounding of a Fraction (nearest, ties to even)."""
+    from fractions import Fraction
+    c = np.float32(float(fr))
+    cands = [np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))]
+    best = None
+    for v in cands:
+        d = abs(Fraction(float(v)) - fr)
+        if best is None or d < best[0] or (d == best[0] and (int(np.float32(v).view(np.uint32)) & 1) == 0):
+            best = (d, v)
+    return best[1]
+
+
+def test_fused_probability_exponent_is_a_single_rounding():
+    # the oracle evaluates fma(S, A, -m) as float64 arithmetic rounded to float32;
+    # check it against exact rational arithmetic over the regimes the path produces
+    from fractions import Fraction
+    rng = np.random.default_rng(19)
+    n_ok = 0
+    for _ in range(3000):
+        S = int(rng.integers(-2_064_512, 2_064_513))
+        A = np.float32(np.exp2(rng.uniform(-30, 0)) * rng.uniform(1, 2))
+        mn = np.float32(rng.choice([1.0, 1e-6, 1e3]) * rng.standard_normal())
+        emu = np.float32(np.float64(S) * np.float64(A) - np.float64(mn))
+        exact = _f32_round_exact(Fraction(S) * Fraction(float(A)) - Fraction(float(mn)))
+        assert emu == exact, (S, A, mn)
+        n_ok += 1
+    assert n_ok == 3000

@@ -87,7 +87,7 @@ struct FwdParams {
 // Columns j with (j % 8) < kPolyPer8 evaluate 2^t with an FMA-pipe polynomial,
 // the rest with the MUFU ex2.approx, so both pipes share the exponentials.
 #ifndef QATTN_POLY_PER8
-#define QATTN_POLY_PER8 0
+#define QATTN_POLY_PER8 2
 #endif
 constexpr int kPolyPer8 = QATTN_POLY_PER8;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: x + kMagic rounds x to an integer
@@ -132,19 +132,6 @@ __device__ __forceinline__ void exp_block(float (&x)[64], float2 a2, float2 nb2)
     x[J] = e.x;
     x[J + 1] = e.y;
     exp_block<J + 2>(x, a2, nb2);
-  }
-}
-
-template <int J>
-__device__ __forceinline__ void exp_block_masked(float (&x)[64], float2 a2, float2 nb2, int nvalid) {
-  if constexpr (J < 64) {
-    float2 t = ffma2(make_float2(x[J], x[J + 1]), a2, nb2);
-    if (J >= nvalid) t.x = -INFINITY;
-    if (J + 1 >= nvalid) t.y = -INFINITY;
-    const float2 e = exp2_pair<J>(t);
-    x[J] = e.x;
-    x[J + 1] = e.y;
-    exp_block_masked<J + 2>(x, a2, nb2, nvalid);
   }
 }
 
@@ -273,7 +260,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint64_t ad = smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          mma_i8_ss(tS, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_i8_ss(tS, ad, bd, C::IDESC_QK, 1u);   // onto the kMagic bits already in S
         }
         tc_commit(s_full + i);
       };
@@ -286,8 +273,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         tc_commit(pv_done + 2 * i + (t & 1));
       };
-      bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ);
-      if (ok) ok = mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV);
+      bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ) &&
+                mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV) &&
+                mbar_wait(s_free + i, 0, abort, p.dev_err, kErrTimeoutS);
       if (ok) {
         tc_fence_after();
         issue_qk(0);
@@ -297,7 +285,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (t + 1 < nK) {
           const int s1 = (t + 1) % C::STAGES;
           ok = mbar_wait(kv_full + s1, ((t + 1) / C::STAGES) & 1, abort, p.dev_err, kErrTimeoutKV) &&
-               mbar_wait(s_free + i, t & 1, abort, p.dev_err, kErrTimeoutS);
+               mbar_wait(s_free + i, (t + 1) & 1, abort, p.dev_err, kErrTimeoutS);
           if (!ok) break;
           tc_fence_after();
           issue_qk(s1);
@@ -330,6 +318,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
       float m = kMInit, den = 1.0f;
       float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
+      // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
+      // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
+      // conversion is needed.  s_free phase t = "S_i reset, QK_i(t) may accumulate".
+      uint32_t magic[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) magic[j] = 0x4B400000u;
+      tmem_st32(tS, magic);
+      tmem_st32(tS + 32, magic);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free + wg);
       bool ok = true;
       for (int t = 0; t < nK; ++t) {
         float ks_cur = ks_next;
@@ -341,13 +341,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + wg);
-        // INT32 score -> FP32 (exact for |S| < 2^22): the bits of kMagic + S, then
-        // minus kMagic (exact)
-#pragma unroll
-        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(__float_as_uint(x[j]) + 0x4B400000u);
+        tmem_st32(tS, magic);                           // reset S for QK_i(t+1)
+        tmem_st32(tS + 32, magic);
         const bool last = (t == nK - 1);
         float mn;
         float2 a2, nb2;
@@ -356,7 +351,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (last) {
 #pragma unroll
             for (int j = 0; j < 64; ++j)
-              if (j >= last_valid) x[j] = 0.0f;          // below every valid kMagic + S
+              if (j >= last_valid) x[j] = -INFINITY;     // masked key: p = 2^-inf = 0
           }
           float mq[4];
 #pragma unroll
@@ -393,20 +388,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const float ksj = (j < nv) ? __half2float(ks16[t * BN + j]) : 0.0f;
-            x[j] = __fmaf_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c), -mn);
+            x[j] = (j < nv) ? __fmaf_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c), -mn) : -INFINITY;
           }
           a2 = make_float2(1.0f, 1.0f);
           nb2 = make_float2(0.0f, 0.0f);
         }
+        tmem_wait_st();                                 // the reset of S has landed
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + wg);
         const float old = ex2_approx(__fsub_rn(m, mn));
         old_s[(wg * 2 + (t & 1)) * BM + row] = old;
         __syncwarp();
         if (lane == 0) mbar_arrive(old_rdy + 2 * wg + (t & 1));
-        if (last) {
-          exp_block_masked<0>(x, a2, nb2, last_valid);
-        } else {
-          exp_block<0>(x, a2, nb2);
-        }
+        exp_block<0>(x, a2, nb2);
         // denominator: unquantized probabilities, four independent pair sums
         float2 acc[4];
 #pragma unroll

@@ -130,6 +130,26 @@ qattn_status qattn_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                   uint16_t* k_scale_f16, uint8_t* v8t, float* v_scale,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Same computation as qattn_quant, for callers that cannot allocate device
+ * memory when they quantize (inside a CUDA-graph capture, under an allocator
+ * that forbids allocation on the hot path, or in an embedder whose memory
+ * manager hands out only the tensors).  The pages have no counterpart: it is
+ * an interface choice of this library, not part of the method.
+ * The scratch lives in one static device array of QATTN_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) compiled into the library; every device that uses the entry point
+ * keeps it until the process exits.  Problems whose qattn_quant_workspace_bytes
+ * exceeds that are refused with QATTN_ERR_WORKSPACE.  All calls share the
+ * array, so calls that overlap on the GPU (other streams or threads) race:
+ * serialize them.  No scratch byte needs clearing between calls.  The first
+ * call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * and caches it; make that first call before any stream capture.
+ * Arguments, layouts and errors otherwise as qattn_quant. */
+#define QATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+qattn_status qattn_quant_noalloc(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                                 qattn_bnhd qp, qattn_bnhd kp, qattn_bnhd v,
+                                 int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                                 float* k_mean, uint8_t* v8t, float* v_scale, void* stream);
+
 /* ---------------------------------------------------------------- fwd
  * Fused attention ("INT8 QK And Score Domain", "Online Softmax", "V And PV",
  * "Finalization And Tails").  Per query row, over 64-key tiles t = 0, 1, ... in

@@ -10,10 +10,11 @@ from __future__ import annotations
 import math
 
 from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_check, qattn_fwd, qattn_prep,  # noqa: F401
-                   qattn_quant, qattn_quant_hadamard, qattn_quant_workspace_bytes, qattn_scores,
-                   qattn_version)
+                   qattn_quant, qattn_quant_hadamard, qattn_quant_noalloc,
+                   qattn_quant_workspace_bytes, qattn_scores, qattn_version)
 
-__all__ = ["Pipeline", "QAttnError", "qattn_prep", "qattn_quant", "qattn_quant_hadamard",
+__all__ = ["Pipeline", "QAttnError", "qattn_prep", "qattn_quant", "qattn_quant_noalloc",
+           "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
            "qattn_version", "load"]
 

@@ -19,7 +19,8 @@ QATTN_STATUS = {0: "QATTN_OK", 1: "QATTN_ERR_NULL", 2: "QATTN_ERR_SHAPE", 3: "QA
                 4: "QATTN_ERR_UNSUPPORTED", 5: "QATTN_ERR_WORKSPACE", 6: "QATTN_ERR_CUDA",
                 7: "QATTN_ERR_TIMEOUT"}
 
-EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_hadamard",
+EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_noalloc",
+            "qattn_quant_hadamard",
             "qattn_fwd", "qattn_scores", "qattn_check", "qattn_last_error", "qattn_version")
 
 
@@ -54,6 +55,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_quant_workspace_bytes.restype = sz
     lib.qattn_quant.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp, vp, vp,
                                 vp, sz, vp]
+    lib.qattn_quant_noalloc.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
+                                        vp, vp, vp]
     lib.qattn_quant_hadamard.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
                                          vp, vp, sz, vp]
     lib.qattn_fwd.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, vp, vp]
@@ -61,7 +64,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_check.argtypes = [vp, vp]
     lib.qattn_last_error.restype = ctypes.c_char_p
     lib.qattn_version.restype = ctypes.c_char_p
-    for name in ("qattn_prep", "qattn_quant", "qattn_quant_hadamard", "qattn_fwd",
+    for name in ("qattn_prep", "qattn_quant", "qattn_quant_noalloc", "qattn_quant_hadamard", "qattn_fwd",
                  "qattn_scores", "qattn_check"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -111,6 +114,14 @@ def qattn_quant(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_m
     _check(load().qattn_quant(B, Nq, Nkv, Hq, Hkv, D, bnhd(qp), bnhd(kp), bnhd(v), _ptr(q8),
                               _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(k_mean), _ptr(v8t),
                               _ptr(v_scale), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def qattn_quant_noalloc(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_mean, v8t,
+                        v_scale, stream=None):
+    """qattn_quant on the library's static scratch (no workspace argument)."""
+    _check(load().qattn_quant_noalloc(B, Nq, Nkv, Hq, Hkv, D, bnhd(qp), bnhd(kp), bnhd(v), _ptr(q8),
+                                      _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(k_mean),
+                                      _ptr(v8t), _ptr(v_scale), _stream(stream)))
 
 
 def qattn_quant_hadamard(B, Nq, Nkv, Hq, Hkv, D, q, k, v, q8, q_scale, k8, k_scale_f16, v8t,

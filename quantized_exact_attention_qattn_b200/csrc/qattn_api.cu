@@ -82,6 +82,8 @@ qattn_status check_sizes(int B, int Nq, int Nkv, int Hq, int Hkv, int D) {
 
 }  // namespace
 
+void qattn::set_last_error(const char* msg) { g_last_error = msg; }
+
 extern "C" {
 
 const char* qattn_version(void) { return "qattn-b200 0.1.0 (sm_100a)"; }

@@ -17,6 +17,9 @@ inline BNHD to_bnhd(const qattn_bnhd& v) {
   return BNHD{static_cast<const uint16_t*>(v.ptr), v.stride[0], v.stride[1], v.stride[2]};
 }
 
+// qattn_api.cu: record the thread-local message returned by qattn_last_error()
+void set_last_error(const char* msg);
+
 // prep.cu
 cudaError_t launch_prep(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD k,
                         const uint16_t* qw, const uint16_t* kw, float eps, int rotary_dim,

@@ -35,6 +35,10 @@ WORKLOAD = {"workload": "canonical interleaved-QKV quantized attention prefill",
             "rotary_dim": 96, "causal": False,
             "l2": "inputs larger than L2 (1.63 GB QKV, 126 MB L2); no flush needed"}
 NOMINAL_FP8_OVER_BF16 = 2.0          # 4.5 / 2.25 PFLOP/s dense (nominal ratio)
+# DRAM bytes per canonical attention launch: ncu dram__bytes_read + write on the
+# B1 N16384 H32 D128 case (303.6 MB) scaled by the units processed (N*H, x4.04).
+# Valid for the attention kernel of commit 0d377b5; None once the kernel changes.
+ATTN_TRAFFIC_BYTES = 1.226e9
 SPEC_FP8_TFLOPS = 4500.0
 
 
@@ -350,7 +354,9 @@ def run_gpu(args):
             "fwd_frac_of_spec_4500": achieved / SPEC_FP8_TFLOPS,
             "prep_quant_ms": ms_step - fwd_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "attn_fwd_kernel<128,2>",
+                         "frac": achieved / peak,
+                         "traffic": ATTN_TRAFFIC_BYTES if args.config == "canonical" else None,
+                         "kernel": "attn_fwd_kernel<128,2>",
                          "peak_source": peak_src,
                          "algorithmic_work": "4*B*H*N^2*D = %.4e ops per launch" % flops},
             "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12,

@@ -37,8 +37,8 @@ WORKLOAD = {"workload": "canonical interleaved-QKV quantized attention prefill",
 NOMINAL_FP8_OVER_BF16 = 2.0          # 4.5 / 2.25 PFLOP/s dense (nominal ratio)
 # DRAM bytes per canonical attention launch: ncu dram__bytes_read + write on the
 # B1 N16384 H32 D128 case (303.6 MB) scaled by the units processed (N*H, x4.04).
-# Valid for the attention kernel of commit 0d377b5; None once the kernel changes.
-ATTN_TRAFFIC_BYTES = 1.226e9
+# Valid only for the attention kernel the capture was taken on; None once it changes.
+ATTN_TRAFFIC_BYTES = None
 SPEC_FP8_TFLOPS = 4500.0
 
 

@@ -420,12 +420,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int j = 0; j < 64; j += 4)
           pk[j / 4] = static_cast<uint32_t>(cvt_e4m3x2(x[j], x[j + 1])) |
                       (static_cast<uint32_t>(cvt_e4m3x2(x[j + 2], x[j + 3])) << 16);
-        if (t >= 2) {   // P buffer (t & 1) was read by PV_i(t-2)
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + (t & 1), ((t >> 1) - 1) & 1,
-                                                 abort, p.dev_err, kErrTimeoutO));
-          if (!ok) break;
-          tc_fence_after();
-        }
+        // P buffer (t & 1) is free: PV_i(t-2) was issued before QK_i(t) by the same
+        // thread, so the commit that signalled s_full(t) covered its completion.
         tmem_st16(tP + (t & 1) * (BN / 4), pk);
         tmem_wait_st();
         tc_fence_before();
@@ -452,32 +448,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ok = __all_sync(0xffffffffu, mbar_wait(old_rdy + 2 * i + (t & 1), (t >> 1) & 1, abort,
                                                p.dev_err, kErrTimeoutO));
         if (!ok) break;
-        if (t > 0) {
+        // A warp whose 32 rows keep their maximum (old == 1) leaves O untouched and
+        // need not wait for PV_i(t-1): the issuing thread orders PV_i(t) after it.
+        const float o = old_s[(i * 2 + (t & 1)) * BM + row];
+        if (t > 0 && __any_sync(0xffffffffu, o != 1.0f)) {
           ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
                                                  abort, p.dev_err, kErrTimeoutO));
           if (!ok) break;
           tc_fence_after();
-          const float o = old_s[(i * 2 + (t & 1)) * BM + row];
-          if (__any_sync(0xffffffffu, o != 1.0f)) {
-            const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
+          const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 64) {
-              uint32_t r[64];
-              tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-              tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-              tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 64) {
+            uint32_t r[64];
+            tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 64; j += 2) {
-                const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
-                                       make_float2(o, o));
-                r[j] = __float_as_uint(v.x);
-                r[j + 1] = __float_as_uint(v.y);
-              }
-              tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-              tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            for (int j = 0; j < 64; j += 2) {
+              const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                     make_float2(o, o));
+              r[j] = __float_as_uint(v.x);
+              r[j + 1] = __float_as_uint(v.y);
             }
-            tmem_wait_st();
+            tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           }
+          tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();

@@ -135,6 +135,13 @@ __device__ __forceinline__ void exp_block(float (&x)[64], float2 a2, float2 nb2)
   }
 }
 
+// Write the kMagic bit pattern into the 64 score columns of this warp's lanes
+// (16 registers hold the pattern: less register pressure than one 32-wide store).
+__device__ __forceinline__ void reset_s(uint32_t tS, const uint32_t (&m)[16]) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 16) tmem_st16(tS + c, m);
+}
+
 template <int D, int NQT, int KMODE>
 __global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -321,11 +328,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
       // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
       // conversion is needed.  s_free phase t = "S_i reset, QK_i(t) may accumulate".
-      uint32_t magic[32];
+      uint32_t magic[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) magic[j] = 0x4B400000u;
-      tmem_st32(tS, magic);
-      tmem_st32(tS + 32, magic);
+      for (int j = 0; j < 16; ++j) magic[j] = 0x4B400000u;
+      reset_s(tS, magic);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -341,8 +347,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
         tmem_wait_ld();
-        tmem_st32(tS, magic);                           // reset S for QK_i(t+1)
-        tmem_st32(tS + 32, magic);
+        reset_s(tS, magic);                             // reset S for QK_i(t+1)
         const bool last = (t == nK - 1);
         float mn;
         float2 a2, nb2;
@@ -417,9 +422,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
         uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 64; j += 4)
-          pk[j / 4] = static_cast<uint32_t>(cvt_e4m3x2(x[j], x[j + 1])) |
-                      (static_cast<uint32_t>(cvt_e4m3x2(x[j + 2], x[j + 3])) << 16);
+        for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
         // P buffer (t & 1) is free: PV_i(t-2) was issued before QK_i(t) by the same
         // thread, so the commit that signalled s_full(t) covered its completion.
         tmem_st16(tP + (t & 1) * (BN / 4), pk);

@@ -55,7 +55,8 @@ struct Cfg {
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
   static constexpr int SMEM_OLD = SMEM_V + STAGES * V_BYTES;        // float [NQT][2][128]
   static constexpr int SMEM_DEN = SMEM_OLD + NQT * 2 * BM * 4;      // float [NQT][128]
-  static constexpr int SMEM_BAR = SMEM_DEN + NQT * BM * 4;
+  static constexpr int SMEM_KS = SMEM_DEN + NQT * BM * 4;           // float [softmax warps][64]
+  static constexpr int SMEM_BAR = SMEM_KS + NQT * 4 * BN * 4;
   static constexpr int N_BARS = 1 + 2 * STAGES + 11 * NQT;
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
   // warps 0-3: producer, one MMA issuer per query tile, spare; then NQT softmax
@@ -152,6 +153,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                              ~static_cast<uintptr_t>(1023));
   float* old_s = reinterpret_cast<float*>(smem + C::SMEM_OLD);     // [NQT][2][BM]
   float* den_s = reinterpret_cast<float*>(smem + C::SMEM_DEN);     // [NQT][BM]
+  float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token K scales
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
@@ -378,23 +380,51 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           a2 = make_float2(a, a);
           nb2 = make_float2(-mn, -mn);
         } else {
-          // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent uses
-          // fma(S_j, A_j, -mn), so x[] keeps S_j and a[] keeps A_j
-          // (A_j is recomputed in the second pass instead of held in registers)
+          // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
+          // fma(S_j, A_j, -mn).  The warp stages the tile's 64 scales in shared
+          // memory (two per lane, one load each) and every thread keeps A_j.
           const int nv = last ? last_valid : BN;
+          float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
+          {
+            const int j0 = 2 * lane;
+            const __half* src = ks16 + t * BN + j0;
+            float k0 = 0.0f, k1 = 0.0f;
+            if (j0 + 1 < nv && (reinterpret_cast<uintptr_t>(src) & 3u) == 0) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(src));
+              k0 = f.x;
+              k1 = f.y;
+            } else {
+              if (j0 < nv) k0 = __half2float(src[0]);
+              if (j0 + 1 < nv) k1 = __half2float(src[1]);
+            }
+            kss[j0] = k0;
+            kss[j0 + 1] = k1;
+          }
+          __syncwarp();
+          // (every lane reads the same address: a broadcast, no bank conflict)
           float smx = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float ksj = (j < nv) ? __half2float(ks16[t * BN + j]) : 0.0f;
-            x[j] = __fsub_rn(x[j], kMagic);
-            if (j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c)));
+          for (int j = 0; j < 64; j += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
+            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              x[j + u] = __fsub_rn(x[j + u], kMagic);
+              if (j + u < nv) smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c)));
+            }
           }
           mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float ksj = (j < nv) ? __half2float(ks16[t * BN + j]) : 0.0f;
-            x[j] = (j < nv) ? __fmaf_rn(x[j], __fmul_rn(__fmul_rn(qs, ksj), p.c), -mn) : -INFINITY;
+          for (int j = 0; j < 64; j += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
+            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              x[j + u] = (j + u < nv)
+                             ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c), -mn)
+                             : -INFINITY;
           }
+          __syncwarp();                                   // kss is rewritten next tile
           a2 = make_float2(1.0f, 1.0f);
           nb2 = make_float2(0.0f, 0.0f);
         }

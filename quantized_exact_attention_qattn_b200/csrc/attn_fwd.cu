@@ -10,18 +10,19 @@
 //
 // Blackwell mapping (one CTA = NQT query tiles of 128 rows of one (b, h)):
 //   warp 0      TMA producer: Q tiles once, then K/V tiles into a STAGES ring
-//   warp 1      tensor-memory owner and single-thread tcgen05.mma issuer:
-//               QK^T as kind::i8 (M=128, N=64, K=32 steps) into TMEM S[i],
-//               P.V as kind::f8f6f4 with P read from TMEM (M=128, N=D, K=32)
-//               accumulating into TMEM O[i]
+//   warp 1+i    single-thread tcgen05.mma issuer of query tile i: QK^T as
+//               kind::i8 (M=128, N=64, K=32 steps) into TMEM S[i] as soon as the
+//               softmax warps have read S[i], then P.V as kind::f8f6f4 with P
+//               read from TMEM (M=128, N=D, K=32) accumulating into TMEM O[i]
 //   warps 4..   one 128-thread softmax warpgroup per query tile; thread r owns
 //               query row r (TMEM lane r): tcgen05.ld of its 64 scores, the
-//               online-softmax update, the O rescale (only when a row's max
-//               moved), tcgen05.st of its 64 FP8 probabilities, and the final
+//               online-softmax update, tcgen05.st of its 64 FP8 probabilities,
+//               the O rescale of its row (only in warps where some row's maximum
+//               moved, after the previous P.V completed), and the final
 //               normalisation + BF16 store.
-// The MMA warp issues PV(i, t) then QK(i, t+1) per tile i, so while one
-// warpgroup runs the softmax of tile t the tensor core works for the other.
-// Every wait is bounded; a timeout sets a device error bit and all roles drain.
+// The two query tiles' chains are independent, so while one warpgroup runs the
+// softmax of its tile the tensor core works for the other.  Every wait is
+// bounded; a timeout sets a device error bit and all roles drain.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -53,17 +54,14 @@ struct Cfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = SMEM_Q + NQT * Q_BYTES;
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
-  static constexpr int SMEM_OLD = SMEM_V + STAGES * V_BYTES;        // float [NQT][2][128]
-  static constexpr int SMEM_DEN = SMEM_OLD + NQT * 2 * BM * 4;      // float [NQT][128]
-  static constexpr int SMEM_KS = SMEM_DEN + NQT * BM * 4;           // float [softmax warps][64]
+  static constexpr int SMEM_KS = SMEM_V + STAGES * V_BYTES;         // float [softmax warps][64]
   static constexpr int SMEM_BAR = SMEM_KS + NQT * 4 * BN * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 11 * NQT;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 7 * NQT;
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
-  // warps 0-3: producer, one MMA issuer per query tile, spare; then NQT softmax
-  // warpgroups; then the correction warpgroup
+  // warps 0-3: producer, one P.V issuer per query tile, spare; then NQT softmax
+  // warpgroups
   static constexpr int SOFTMAX_WARP0 = 4;
-  static constexpr int CORR_WARP0 = 4 + 4 * NQT;
-  static constexpr int THREADS = 32 * (CORR_WARP0 + 4);
+  static constexpr int THREADS = 32 * (SOFTMAX_WARP0 + 4 * NQT);
   // tensor memory columns: O[NQT] (D each), S[NQT] (64 each), P[NQT][2] (16 each)
   static constexpr uint32_t O_COL = 0;
   static constexpr uint32_t S_COL = NQT * D;
@@ -138,6 +136,27 @@ __device__ __forceinline__ void exp_block(float (&x)[64], float2 a2, float2 nb2)
 
 // Write the kMagic bit pattern into the 64 score columns of this warp's lanes
 // (16 registers hold the pattern: less register pressure than one 32-wide store).
+// O <- O * o for this warp's 32 rows of O (tensor memory), 64 columns at a time.
+template <int D>
+__device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 64) {
+    uint32_t r[64];
+    tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 64; j += 2) {
+      const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                             make_float2(o, o));
+      r[j] = __float_as_uint(v.x);
+      r[j + 1] = __float_as_uint(v.y);
+    }
+    tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  }
+}
+
 __device__ __forceinline__ void reset_s(uint32_t tS, const uint32_t (&m)[16]) {
 #pragma unroll
   for (int c = 0; c < 64; c += 16) tmem_st16(tS + c, m);
@@ -151,25 +170,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* old_s = reinterpret_cast<float*>(smem + C::SMEM_OLD);     // [NQT][2][BM]
-  float* den_s = reinterpret_cast<float*>(smem + C::SMEM_DEN);     // [NQT][BM]
   float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token K scales
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  // A parity wait for phase k is only sound if phase k+1 cannot complete before
-  // the waiter is through.  Where the producer side could run two phases ahead
-  // (rescale factors, P buffers and the P.V products that read them) there is
-  // one barrier per buffer, indexed [i][t & 1]; every other barrier's next phase
-  // depends on its waiter having passed (checked per barrier below).
+  // A parity wait for phase k is only sound if phase k-1 has completed and phase
+  // k+1 cannot complete before the waiter is through.  P buffers, P-full and
+  // PV-done are replicated per tile parity, [i][t & 1]: softmax writes P_i(t+2)
+  // only after PV_i(t+1) (and so PV_i(t)) completed, PV_i(t+2) needs P_i(t+2),
+  // and every waiter waits for every phase in order.  Every other barrier's next
+  // phase depends on its waiter having passed.
   uint64_t* s_full = kv_empty + C::STAGES;   // MMA -> softmax: S_i(t) in TMEM
-  uint64_t* s_free = s_full + NQT;           // softmax -> MMA: S_i(t) read
-  uint64_t* o_rdy = s_free + NQT;            // correction -> MMA: O_i rescaled for t
-  uint64_t* fin = o_rdy + NQT;               // softmax -> correction: final denominators
-  uint64_t* old_rdy = fin + NQT;             // [NQT][2] softmax -> correction: old(t) in smem
-  uint64_t* p_full = old_rdy + 2 * NQT;      // [NQT][2] softmax -> MMA: P_i(t) in TMEM
-  uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax/correction: PV_i(t) done
+  uint64_t* s_free = s_full + NQT;           // softmax -> MMA: S_i read and reset
+  uint64_t* p_full = s_free + NQT;           // [NQT][2] softmax -> MMA: P_i(t) written, O_i rescaled
+  uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax: PV_i(t) done
   uint64_t* drain = pv_done + 2 * NQT;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -193,19 +208,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(q_full, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, nvalid);      // one commit per MMA issuer
+      mbar_init(kv_empty + s, nvalid);      // one commit per P.V issuer
     }
     for (int i = 0; i < NQT; ++i) {
       mbar_init(s_full + i, 1);
-      // arrivals from softmax / correction warpgroups: one elected lane per warp
-      mbar_init(s_free + i, 4);
-      mbar_init(o_rdy + i, 4);
-      mbar_init(fin + i, 4);
       for (int bb = 0; bb < 2; ++bb) {
-        mbar_init(old_rdy + 2 * i + bb, 4);
-        mbar_init(p_full + 2 * i + bb, 4);
+        mbar_init(p_full + 2 * i + bb, 4);    // one elected lane per softmax warp
         mbar_init(pv_done + 2 * i + bb, 1);
       }
+      mbar_init(s_free + i, 4);
     }
     for (int i = 0; i < NQT; ++i) mbar_init(drain + i, 1);
     fence_barrier_init();
@@ -254,7 +265,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ================================================================ MMA issuers
     // One issuing thread per query tile i (warp 1 + i), so the two tiles' chains
     // never wait on each other: QK_i(t+1) as soon as S_i(t) has been read, then
-    // PV_i(t) once P_i(t) is written and O_i rescaled.
+    // PV_i(t) once the softmax warps have written P_i(t) and rescaled O_i.
     const int i = warp - 1;
     if (lane == 0 && i < nvalid) {
       const uint32_t sQ = smem_u32(smem + C::SMEM_Q) + i * C::Q_BYTES;
@@ -273,15 +284,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         tc_commit(s_full + i);
       };
-      auto issue_pv = [&](int s, int t) {
-        const uint32_t a_tm = tmem + C::P_COL + (i * 2 + (t & 1)) * (BN / 4);
-#pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk) {
-          const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
-          mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(pv_done + 2 * i + (t & 1));
-      };
       bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ) &&
                 mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV) &&
                 mbar_wait(s_free + i, 0, abort, p.dev_err, kErrTimeoutS);
@@ -299,11 +301,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           issue_qk(s1);
         }
-        ok = mbar_wait(p_full + 2 * i + (t & 1), (t >> 1) & 1, abort, p.dev_err, kErrTimeoutP) &&
-             mbar_wait(o_rdy + i, t & 1, abort, p.dev_err, kErrTimeoutO);
+        ok = mbar_wait(p_full + 2 * i + (t & 1), (t >> 1) & 1, abort, p.dev_err, kErrTimeoutP);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(s, t);
+        const uint32_t a_tm = tmem + C::P_COL + (i * 2 + (t & 1)) * (BN / 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 32; ++kk) {
+          const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
+          mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(pv_done + 2 * i + (t & 1));
         tc_commit(kv_empty + s);   // stage s is free once every issuer's reads finished
       }
       tc_commit(drain + i);        // drain: every issued tensor-core op before tear-down
@@ -311,7 +318,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_wait(drain + i, 0, &dummy, p.dev_err, kErrTimeoutDrain);
     }
     __syncwarp();
-  } else if (warp >= C::SOFTMAX_WARP0 && warp < C::CORR_WARP0) {
+  } else if (warp >= C::SOFTMAX_WARP0) {
     // ================================================================ softmax
     const int wg = (warp - C::SOFTMAX_WARP0) >> 2;
     const int q4 = warp & 3;
@@ -321,15 +328,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
       const uint32_t tS = tmem + lane_off + C::S_COL + wg * BN;
       const uint32_t tP = tmem + lane_off + C::P_COL + (wg * 2) * (BN / 4);
+      const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
       const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
       const int last_valid = p.Nkv - (nK - 1) * BN;
       const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
       const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
       float m = kMInit, den = 1.0f;
       float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
+      // per-token scales: lane l holds tokens 2l, 2l+1 of a tile (0 past the end)
+      auto load_kpair = [&](int tt) {
+        const int j = tt * BN + 2 * lane;
+        return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
+                           j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+      };
+      float2 kpair_next = make_float2(0.0f, 0.0f);
+      if constexpr (KMODE == 1) kpair_next = load_kpair(0);
       // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
       // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
-      // conversion is needed.  s_free phase t = "S_i reset, QK_i(t) may accumulate".
+      // conversion is needed.
       uint32_t magic[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) magic[j] = 0x4B400000u;
@@ -337,11 +353,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + wg);
+      if (lane == 0) mbar_arrive(s_free + wg);      // s_free phase t: QK_i(t) may accumulate
       bool ok = true;
-      for (int t = 0; t < nK; ++t) {
+      for (int t = 0; ok && t < nK; ++t) {
         float ks_cur = ks_next;
         if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
+        const float2 kpair = kpair_next;
+        if constexpr (KMODE == 1) {
+          if (t + 1 < nK) kpair_next = load_kpair(t + 1);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
         if (!ok) break;
         tc_fence_after();
@@ -385,21 +405,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // memory (two per lane, one load each) and every thread keeps A_j.
           const int nv = last ? last_valid : BN;
           float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
-          {
-            const int j0 = 2 * lane;
-            const __half* src = ks16 + t * BN + j0;
-            float k0 = 0.0f, k1 = 0.0f;
-            if (j0 + 1 < nv && (reinterpret_cast<uintptr_t>(src) & 3u) == 0) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(src));
-              k0 = f.x;
-              k1 = f.y;
-            } else {
-              if (j0 < nv) k0 = __half2float(src[0]);
-              if (j0 + 1 < nv) k1 = __half2float(src[1]);
-            }
-            kss[j0] = k0;
-            kss[j0 + 1] = k1;
-          }
+          kss[2 * lane] = kpair.x;                      // this tile's scales, fetched a tile ago
+          kss[2 * lane + 1] = kpair.y;
           __syncwarp();
           // (every lane reads the same address: a broadcast, no bank conflict)
           float smx = -INFINITY;
@@ -433,9 +440,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free + wg);
         const float old = ex2_approx(__fsub_rn(m, mn));
-        old_s[(wg * 2 + (t & 1)) * BM + row] = old;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(old_rdy + 2 * wg + (t & 1));
         exp_block<0>(x, a2, nb2);
         // denominator: unquantized probabilities, four independent pair sums
         float2 acc[4];
@@ -453,99 +457,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
-        // P buffer (t & 1) is free: PV_i(t-2) was issued before QK_i(t) by the same
-        // thread, so the commit that signalled s_full(t) covered its completion.
-        tmem_st16(tP + (t & 1) * (BN / 4), pk);
-        tmem_wait_st();
-        tc_fence_before();
-        if (last) den_s[wg * BM + row] = den;
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(p_full + 2 * wg + (t & 1));
-          if (last) mbar_arrive(fin + wg);
-        }
-        m = mn;
-      }
-      (void)ok;
-    }
-  } else if (warp >= C::CORR_WARP0) {
-    // ================================================================ correction
-    // Rescales O_i by old(t) between PV_i(t-1) and PV_i(t) (only warps in which
-    // some row's maximum moved), then normalises and stores the output.
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    bool ok = true;
-    for (int t = 0; ok && t < nK; ++t) {
-      for (int i = 0; i < nvalid; ++i) {
-        ok = __all_sync(0xffffffffu, mbar_wait(old_rdy + 2 * i + (t & 1), (t >> 1) & 1, abort,
-                                               p.dev_err, kErrTimeoutO));
-        if (!ok) break;
-        // A warp whose 32 rows keep their maximum (old == 1) leaves O untouched and
-        // need not wait for PV_i(t-1): the issuing thread orders PV_i(t) after it.
-        const float o = old_s[(i * 2 + (t & 1)) * BM + row];
-        if (t > 0 && __any_sync(0xffffffffu, o != 1.0f)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
+        if (t >= 1) {
+          // PV_i(t-1) was issued when this warpgroup finished tile t-1 and has long
+          // completed.  Its completion frees P buffer (t & 1), last read by
+          // PV_i(t-2), and lets this warp rescale its rows of O_i by old before
+          // PV_i(t) accumulates (only if one of its 32 rows' maximum moved).
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((t - 1) & 1), ((t - 1) >> 1) & 1,
                                                  abort, p.dev_err, kErrTimeoutO));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            uint32_t r[64];
-            tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 64; j += 2) {
-              const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
-                                     make_float2(o, o));
-              r[j] = __float_as_uint(v.x);
-              r[j + 1] = __float_as_uint(v.y);
-            }
-            tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          }
-          tmem_wait_st();
+          if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D>(tO, old);
         }
+        tmem_st16(tP + (t & 1) * (BN / 4), pk);
+        tmem_wait_st();                                 // P and any O rescale have landed
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(o_rdy + i);
+        if (lane == 0) mbar_arrive(p_full + 2 * wg + (t & 1));
+        m = mn;
       }
-    }
-    // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only
-    for (int i = 0; ok && i < nvalid; ++i) {
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(pv_done + 2 * i + ((nK - 1) & 1), ((nK - 1) >> 1) & 1, abort,
-                                p.dev_err, kErrTimeoutO) &&
-                          mbar_wait(fin + i, 0, abort, p.dev_err, kErrTimeoutO));
-      if (!ok) break;
-      tc_fence_after();
-      const float inv = rcp_approx(den_s[i * BM + row]);
-      const int n = (qt0 + i) * BM + row;
-      const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
-      uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
-      const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
+      // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization")
+      if (ok)
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
+                                               abort, p.dev_err, kErrTimeoutO));
+      if (ok) {
+        tc_fence_after();
+        const float inv = rcp_approx(den);
+        const int n = qt * BM + row;
+        const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
+        uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + c0, o);
-        tmem_wait_ld();
-        if (n < p.Nq) {
-          uint32_t w[16];
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld();
+          if (n < p.Nq) {
+            uint32_t w[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                         make_float2(inv, inv)),
-                                   make_float2(vs[c0 + j], vs[c0 + j + 1]));
-            w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                       (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                           make_float2(inv, inv)),
+                                     make_float2(vs[c0 + j], vs[c0 + j + 1]));
+              w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+            d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-          d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-          d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
         }
       }
     }

@@ -14,12 +14,16 @@
 //               kind::i8 (M=128, N=64, K=32 steps) into TMEM S[i] as soon as the
 //               softmax warps have read S[i], then P.V as kind::f8f6f4 with P
 //               read from TMEM (M=128, N=D, K=32) accumulating into TMEM O[i]
-//   warps 4..   one 128-thread softmax warpgroup per query tile; thread r owns
-//               query row r (TMEM lane r): tcgen05.ld of its 64 scores, the
-//               online-softmax update, tcgen05.st of its 64 FP8 probabilities,
-//               the O rescale of its row (only in warps where some row's maximum
-//               moved, after the previous P.V completed), and the final
-//               normalisation + BF16 store.
+//   warps 4..   D <= 128: one 128-thread softmax warpgroup per query tile;
+//               thread r owns query row r (TMEM lane r): tcgen05.ld of its 64
+//               scores, the online-softmax update, tcgen05.st of its 64 FP8
+//               probabilities, the O rescale of its row (only in warps where some
+//               row's maximum moved, after the previous P.V completed), and the
+//               final normalisation + BF16 store.
+//   warps 3..   D = 256: two warpgroups per query tile, one per half of the 64
+//               keys (and of the O columns); the two warps on the same rows swap
+//               their half-row maxima through shared memory every tile, and add
+//               their partial denominators at the end.
 // The two query tiles' chains are independent, so while one warpgroup runs the
 // softmax of its tile the tensor core works for the other.  Every wait is
 // bounded; a timeout sets a device error bit and all roles drain.
@@ -54,14 +58,24 @@ struct Cfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = SMEM_Q + NQT * Q_BYTES;
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
-  static constexpr int SMEM_KS = SMEM_V + STAGES * V_BYTES;         // float [softmax warps][64]
-  static constexpr int SMEM_BAR = SMEM_KS + NQT * 4 * BN * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 7 * NQT;
+  // Softmax layout: one warpgroup per query tile owning whole 64-key rows, or (for
+  // D = 256, where the longer P.V gives the softmax more time per tile and more
+  // warps hide more of its latency) two per query tile, one per half of the keys.
+  static constexpr bool SPLIT = (D == 256);
+  static constexpr int SM_WARPS = (SPLIT ? 8 : 4) * NQT;            // softmax warps
+  static constexpr int ARRIVALS = SPLIT ? 8 : 4;                    // softmax warps per query tile
+  static constexpr int KS_PER_WARP = SPLIT ? 32 : 64;               // staged per-token K scales
+  static constexpr int SMEM_KS = SMEM_V + STAGES * V_BYTES;         // float [softmax warps][KS_PER_WARP]
+  static constexpr int SMEM_DEN = SMEM_KS + SM_WARPS * KS_PER_WARP * 4;  // float [NQT][2][128]
+  static constexpr int SMEM_PMAX = SMEM_DEN + NQT * 2 * BM * 4;     // float [NQT][2][2][128]
+  static constexpr int SMEM_BAR = SMEM_PMAX + NQT * 4 * BM * 4;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 11 * NQT;
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
-  // warps 0-3: producer, one P.V issuer per query tile, spare; then NQT softmax
-  // warpgroups
-  static constexpr int SOFTMAX_WARP0 = 4;
-  static constexpr int THREADS = 32 * (SOFTMAX_WARP0 + 4 * NQT);
+  // warps 0..: producer, one MMA issuer per query tile (then a spare warp or two),
+  // then the softmax warps; any four consecutive warps cover the four TMEM lane
+  // quadrants (warp % 4)
+  static constexpr int SOFTMAX_WARP0 = SPLIT ? 3 : 4;
+  static constexpr int THREADS = 32 * (SOFTMAX_WARP0 + SM_WARPS);
   // tensor memory columns: O[NQT] (D each), S[NQT] (64 each), P[NQT][2] (16 each)
   static constexpr uint32_t O_COL = 0;
   static constexpr uint32_t S_COL = NQT * D;
@@ -122,44 +136,48 @@ __device__ __forceinline__ float2 exp2_pair(float2 t) {
   }
 }
 
-// x[j] holds the exact FP32 score S_j; the exponent is fma(S_j, A, -mn).
-template <int J>
-__device__ __forceinline__ void exp_block(float (&x)[64], float2 a2, float2 nb2) {
-  if constexpr (J < 64) {
+// x[j] holds the exact FP32 score S_j; the exponent is fma(S_j, A, -mn).  Columns
+// J .. END-1 of the row's N values, two at a time.
+template <int J, int END, int N>
+__device__ __forceinline__ void exp_block(float (&x)[N], float2 a2, float2 nb2) {
+  if constexpr (J < END) {
     const float2 t = ffma2(make_float2(x[J], x[J + 1]), a2, nb2);
     const float2 e = exp2_pair<J>(t);
     x[J] = e.x;
     x[J + 1] = e.y;
-    exp_block<J + 2>(x, a2, nb2);
+    exp_block<J + 2, END>(x, a2, nb2);
   }
 }
 
-// Write the kMagic bit pattern into the 64 score columns of this warp's lanes
-// (16 registers hold the pattern: less register pressure than one 32-wide store).
-// O <- O * o for this warp's 32 rows of O (tensor memory), 64 columns at a time.
-template <int D>
+// S <- kMagic bits for this warp's 32 rows, 64 columns (four 16-column stores).
+__device__ __forceinline__ void reset_s(uint32_t tS, const uint32_t (&m)[16]) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 16) tmem_st16(tS + c, m);
+}
+
+// O <- O * o for this warp's 32 rows and NCOL columns of O (tensor memory), 64
+// (or, for a 32-column block, 32) columns at a time.
+template <int NCOL>
 __device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
+  constexpr int CH = (NCOL % 64 == 0) ? 64 : 32;
 #pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 64) {
-    uint32_t r[64];
-    tmem_ld32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    tmem_ld32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  for (int c0 = 0; c0 < NCOL; c0 += CH) {
+    uint32_t r[CH];
+#pragma unroll
+    for (int c = 0; c < CH; c += 32)
+      tmem_ld32(tO + c0 + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 64; j += 2) {
+    for (int j = 0; j < CH; j += 2) {
       const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
                              make_float2(o, o));
       r[j] = __float_as_uint(v.x);
       r[j + 1] = __float_as_uint(v.y);
     }
-    tmem_st32(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    tmem_st32(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-  }
-}
-
-__device__ __forceinline__ void reset_s(uint32_t tS, const uint32_t (&m)[16]) {
 #pragma unroll
-  for (int c = 0; c < 64; c += 16) tmem_st16(tS + c, m);
+    for (int c = 0; c < CH; c += 32)
+      tmem_st32(tO + c0 + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
+  }
 }
 
 template <int D, int NQT, int KMODE>
@@ -171,6 +189,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token K scales
+  float* den_s = reinterpret_cast<float*>(smem + C::SMEM_DEN);     // partial denominators
+  float* pmax_s = reinterpret_cast<float*>(smem + C::SMEM_PMAX);   // half-row tile maxima
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
@@ -186,6 +206,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* p_full = s_free + NQT;           // [NQT][2] softmax -> MMA: P_i(t) written, O_i rescaled
   uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax: PV_i(t) done
   uint64_t* drain = pv_done + 2 * NQT;
+  uint64_t* pair_bar = drain + NQT;          // [NQT][4] the two halves of a row quadrant: tile maximum
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -213,10 +234,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int i = 0; i < NQT; ++i) {
       mbar_init(s_full + i, 1);
       for (int bb = 0; bb < 2; ++bb) {
-        mbar_init(p_full + 2 * i + bb, 4);    // one elected lane per softmax warp
+        mbar_init(p_full + 2 * i + bb, C::ARRIVALS);   // one lane per softmax warp
         mbar_init(pv_done + 2 * i + bb, 1);
       }
-      mbar_init(s_free + i, 4);
+      mbar_init(s_free + i, C::ARRIVALS);             // one lane per softmax warp
+      for (int q = 0; q < 4; ++q) mbar_init(pair_bar + i * 4 + q, 2);
     }
     for (int i = 0; i < NQT; ++i) mbar_init(drain + i, 1);
     fence_barrier_init();
@@ -319,192 +341,423 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     __syncwarp();
   } else if (warp >= C::SOFTMAX_WARP0) {
-    // ================================================================ softmax
-    const int wg = (warp - C::SOFTMAX_WARP0) >> 2;
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
-    if (wg < nvalid) {
-      const int qt = qt0 + wg;
+    if constexpr (C::SPLIT) {
+      // ================================================================ softmax
+      // Two warpgroups per query tile i, one per half hf of the 64 key columns
+      // (warpgroup g = 2 i + hf).  Thread r of either owns query row r (TMEM lane r):
+      // both read all 64 scores for the tile maximum, each exponentiates, converts
+      // and stores its own 32, keeps its own partial denominator, and rescales and
+      // normalises its own half of the O columns.
+      const int g = (warp - C::SOFTMAX_WARP0) >> 2;
+      const int i = g >> 1, hf = g & 1;
+      const int q4 = warp & 3;
+      const int row = q4 * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-      const uint32_t tS = tmem + lane_off + C::S_COL + wg * BN;
-      const uint32_t tP = tmem + lane_off + C::P_COL + (wg * 2) * (BN / 4);
-      const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
-      const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
-      const int last_valid = p.Nkv - (nK - 1) * BN;
-      const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
-      const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
-      float m = kMInit, den = 1.0f;
-      float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
-      // per-token scales: lane l holds tokens 2l, 2l+1 of a tile (0 past the end)
-      auto load_kpair = [&](int tt) {
-        const int j = tt * BN + 2 * lane;
-        return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
-                           j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
-      };
-      float2 kpair_next = make_float2(0.0f, 0.0f);
-      if constexpr (KMODE == 1) kpair_next = load_kpair(0);
-      // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
-      // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
-      // conversion is needed.
-      uint32_t magic[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) magic[j] = 0x4B400000u;
-      reset_s(tS, magic);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + wg);      // s_free phase t: QK_i(t) may accumulate
+      const uint32_t tO = tmem + lane_off + C::O_COL + i * D + hf * (D / 2);
       bool ok = true;
-      for (int t = 0; ok && t < nK; ++t) {
-        float ks_cur = ks_next;
-        if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
-        const float2 kpair = kpair_next;
-        if constexpr (KMODE == 1) {
-          if (t + 1 < nK) kpair_next = load_kpair(t + 1);
-        }
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
-        if (!ok) break;
-        tc_fence_after();
-        float x[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tmem_wait_ld();
-        reset_s(tS, magic);                             // reset S for QK_i(t+1)
-        const bool last = (t == nK - 1);
-        float mn;
-        float2 a2, nb2;
-        if constexpr (KMODE == 0) {
-          // A = (q_scale * k_scale) * c; tile max of S*A from the max of S (A > 0)
-          if (last) {
+      float den = (hf == 0) ? 1.0f : 0.0f;   // the two halves' partial sums add up to d
+      if (i < nvalid) {
+        const int qt = qt0 + i;
+        const uint32_t tS = tmem + lane_off + C::S_COL + i * BN;
+        const uint32_t tS_own = tS + hf * 32;
+        const uint32_t tP = tmem + lane_off + C::P_COL + (i * 2) * (BN / 4) + hf * (BN / 8);
+        const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
+        const int last_valid = p.Nkv - (nK - 1) * BN;
+        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
+        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
+        float m = kMInit;
+        float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
+        // per-token scales: lane l holds token 32 hf + l of a tile (0 past the end)
+        auto load_kone = [&](int tt) {
+          const int j = tt * BN + hf * 32 + lane;
+          return j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f;
+        };
+        float kone_next = 0.0f;
+        if constexpr (KMODE == 1) kone_next = load_kone(0);
+        // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
+        // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
+        // conversion is needed.  Each half resets its own 32 columns.
+        uint32_t magic[8];
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-              if (j >= last_valid) x[j] = -INFINITY;     // masked key: p = 2^-inf = 0
-          }
-          float mq[4];
+        for (int j = 0; j < 8; ++j) magic[j] = 0x4B400000u;
+        auto reset_own = [&]() {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            mq[q] = x[16 * q];
-#pragma unroll
-            for (int j = 1; j < 16; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
-          }
-          const float xmax = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
-#pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
-            x[j] = sj.x;
-            x[j + 1] = sj.y;
-          }
-          const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-          const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
-          mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
-          a2 = make_float2(a, a);
-          nb2 = make_float2(-mn, -mn);
-        } else {
-          // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
-          // fma(S_j, A_j, -mn).  The warp stages the tile's 64 scales in shared
-          // memory (two per lane, one load each) and every thread keeps A_j.
-          const int nv = last ? last_valid : BN;
-          float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
-          kss[2 * lane] = kpair.x;                      // this tile's scales, fetched a tile ago
-          kss[2 * lane + 1] = kpair.y;
-          __syncwarp();
-          // (every lane reads the same address: a broadcast, no bank conflict)
-          float smx = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 64; j += 4) {
-            const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
-            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              x[j + u] = __fsub_rn(x[j + u], kMagic);
-              if (j + u < nv) smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c)));
-            }
-          }
-          mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
-#pragma unroll
-          for (int j = 0; j < 64; j += 4) {
-            const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
-            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              x[j + u] = (j + u < nv)
-                             ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c), -mn)
-                             : -INFINITY;
-          }
-          __syncwarp();                                   // kss is rewritten next tile
-          a2 = make_float2(1.0f, 1.0f);
-          nb2 = make_float2(0.0f, 0.0f);
-        }
-        tmem_wait_st();                                 // the reset of S has landed
+          for (int c = 0; c < 32; c += 8) tmem_st8(tS_own + c, magic);
+        };
+        reset_own();
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + wg);
-        const float old = ex2_approx(__fsub_rn(m, mn));
-        exp_block<0>(x, a2, nb2);
-        // denominator: unquantized probabilities, four independent pair sums
-        float2 acc[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
-#pragma unroll
-        for (int j = 8; j < 64; j += 8) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
-        }
-        acc[0] = fadd2(acc[0], acc[1]);
-        acc[2] = fadd2(acc[2], acc[3]);
-        acc[0] = fadd2(acc[0], acc[2]);
-        den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
-        if (t >= 1) {
-          // PV_i(t-1) was issued when this warpgroup finished tile t-1 and has long
-          // completed.  Its completion frees P buffer (t & 1), last read by
-          // PV_i(t-2), and lets this warp rescale its rows of O_i by old before
-          // PV_i(t) accumulates (only if one of its 32 rows' maximum moved).
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((t - 1) & 1), ((t - 1) >> 1) & 1,
-                                                 abort, p.dev_err, kErrTimeoutO));
+        if (lane == 0) mbar_arrive(s_free + i);       // s_free phase t: QK_i(t) may accumulate
+        for (int t = 0; ok && t < nK; ++t) {
+          const float ks_cur = ks_next;
+          if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
+          const float kone = kone_next;
+          if constexpr (KMODE == 1) {
+            if (t + 1 < nK) kone_next = load_kone(t + 1);
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, t & 1, abort, p.dev_err, kErrTimeoutS));
           if (!ok) break;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D>(tO, old);
-        }
-        tmem_st16(tP + (t & 1) * (BN / 4), pk);
-        tmem_wait_st();                                 // P and any O rescale have landed
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + 2 * wg + (t & 1));
-        m = mn;
-      }
-      // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization")
-      if (ok)
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
-                                               abort, p.dev_err, kErrTimeoutO));
-      if (ok) {
-        tc_fence_after();
-        const float inv = rcp_approx(den);
-        const int n = qt * BM + row;
-        const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
-        uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c0, o);
+          float x[32];                                    // this half's 32 scores
+          tmem_ld32(tS_own, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
           tmem_wait_ld();
-          if (n < p.Nq) {
-            uint32_t w[16];
+          reset_own();                                    // reset S for QK_i(t+1)
+          const bool last = (t == nK - 1);
+          const int nv = last ? last_valid : BN;          // valid keys in this tile
+          const int own0 = hf * 32;                       // first key of this half
+          // The row's maximum over both halves: exchanged with the partner warp (same
+          // rows, other half) through shared memory, one slot per tile parity, behind a
+          // two-arrival mbarrier (a bounded wait).  Both warps then hold the same
+          // maximum, so both compute the same mn and old.
+          float* my_max = pmax_s + ((i * 2 + (t & 1)) * 2 + hf) * BM + row;
+          const float* their_max = pmax_s + ((i * 2 + (t & 1)) * 2 + (1 - hf)) * BM + row;
+          bool pair_ok = true;
+          auto pair_max = [&](float v) {
+            *my_max = v;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar + i * 4 + q4);
+            pair_ok = __all_sync(0xffffffffu, mbar_wait(pair_bar + i * 4 + q4, t & 1, abort, p.dev_err,
+                                                        kErrTimeoutS));
+            return fmaxf(v, *their_max);
+          };
+          float mn;
+          float2 a2, nb2;
+          if constexpr (KMODE == 0) {
+            // A = (q_scale * k_scale) * c; tile max of S*A from the max of S (A > 0)
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (own0 + j >= nv) x[j] = -INFINITY;     // masked key: p = 2^-inf = 0
+            }
+            // two independent chains over 16 values each: 7 three-input maxima + 1
+            float mq[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              mq[q] = fmaxf(x[16 * q], x[16 * q + 15]);
+#pragma unroll
+              for (int j = 1; j < 15; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
+            }
+            const float xmax = pair_max(fmaxf(mq[0], mq[1]));
+            if (!pair_ok) {
+              ok = false;
+              break;
+            }
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                           make_float2(inv, inv)),
-                                     make_float2(vs[c0 + j], vs[c0 + j + 1]));
-              w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
             }
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-            d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
+            a2 = make_float2(a, a);
+            nb2 = make_float2(-mn, -mn);
+          } else {
+            // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
+            // fma(S_j, A_j, -mn).  The warp stages its half's 32 scales in shared
+            // memory (one per lane); every lane reads them all (broadcasts).
+            float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * 32;
+            kss[lane] = kone;                             // this tile's scale, fetched a tile ago
+            __syncwarp();
+            float smx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 km = *reinterpret_cast<const float4*>(kss + j);
+              const float kkm[4] = {km.x, km.y, km.z, km.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                x[j + u] = __fsub_rn(x[j + u], kMagic);
+                if (own0 + j + u < nv)
+                  smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kkm[u]), p.c)));
+              }
+            }
+            mn = fmaxf(m, __fsub_rn(pair_max(smx), kFp8Offset));
+            if (!pair_ok) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 km = *reinterpret_cast<const float4*>(kss + j);
+              const float kkm[4] = {km.x, km.y, km.z, km.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                x[j + u] = (own0 + j + u < nv)
+                               ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kkm[u]), p.c), -mn)
+                               : -INFINITY;
+            }
+            __syncwarp();                                   // kss is rewritten next tile
+            a2 = make_float2(1.0f, 1.0f);
+            nb2 = make_float2(0.0f, 0.0f);
+          }
+          tmem_wait_st();                                 // the reset of S has landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + i);
+          const float old = ex2_approx(__fsub_rn(m, mn));
+          exp_block<0, 32>(x, a2, nb2);
+          // partial denominator: unquantized probabilities, four independent pair sums
+          float2 acc[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
+#pragma unroll
+          for (int j = 8; j < 32; j += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
+          }
+          acc[0] = fadd2(acc[0], acc[1]);
+          acc[2] = fadd2(acc[2], acc[3]);
+          acc[0] = fadd2(acc[0], acc[2]);
+          den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+          if (t >= 1) {
+            // PV_i(t-1) was issued when both halves finished tile t-1 and has long
+            // completed.  Its completion frees P buffer (t & 1), last read by
+            // PV_i(t-2), and lets this warp rescale its rows and half of O_i by
+            // old before PV_i(t) accumulates (only if some row's maximum moved).
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
+                                                   abort, p.dev_err, kErrTimeoutO));
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D / 2>(tO, old);
+          }
+          tmem_st8(tP + (t & 1) * (BN / 4), pk);
+          tmem_wait_st();                                 // P and any O rescale have landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + 2 * i + (t & 1));
+          m = mn;
+        }
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
+                                                 abort, p.dev_err, kErrTimeoutO));
+        // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization").
+        // The two halves exchange partial denominators; d = d_0 + d_1 on both.
+        den_s[(i * 2 + hf) * BM + row] = den;
+        const bool any_failed = named_bar_red_or(9 + i, 256, !ok);
+        if (!any_failed) {
+          tc_fence_after();
+          const float inv = rcp_approx(__fadd_rn(den_s[(i * 2) * BM + row], den_s[(i * 2 + 1) * BM + row]));
+          const int n = qt * BM + row;
+          const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D + hf * (D / 2);
+          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + hf * (D / 2);
+#pragma unroll 1
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_wait_ld();
+            if (n < p.Nq) {
+              uint32_t w[16];
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                             make_float2(inv, inv)),
+                                       make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+              }
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+              d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+              d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            }
+          }
+        }
+      }
+    } else {
+      // ================================================================ softmax
+      const int wg = (warp - C::SOFTMAX_WARP0) >> 2;
+      const int q4 = warp & 3;
+      const int row = q4 * 32 + lane;
+      if (wg < nvalid) {
+        const int qt = qt0 + wg;
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::S_COL + wg * BN;
+        const uint32_t tP = tmem + lane_off + C::P_COL + (wg * 2) * (BN / 4);
+        const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
+        const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
+        const int last_valid = p.Nkv - (nK - 1) * BN;
+        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
+        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
+        float m = kMInit, den = 1.0f;
+        float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
+        // per-token scales: lane l holds tokens 2l, 2l+1 of a tile (0 past the end)
+        auto load_kpair = [&](int tt) {
+          const int j = tt * BN + 2 * lane;
+          return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
+                             j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+        };
+        float2 kpair_next = make_float2(0.0f, 0.0f);
+        if constexpr (KMODE == 1) kpair_next = load_kpair(0);
+        // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
+        // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
+        // conversion is needed.
+        uint32_t magic[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) magic[j] = 0x4B400000u;
+        reset_s(tS, magic);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + wg);      // s_free phase t: QK_i(t) may accumulate
+        bool ok = true;
+        for (int t = 0; ok && t < nK; ++t) {
+          float ks_cur = ks_next;
+          if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
+          const float2 kpair = kpair_next;
+          if constexpr (KMODE == 1) {
+            if (t + 1 < nK) kpair_next = load_kpair(t + 1);
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
+          if (!ok) break;
+          tc_fence_after();
+          float x[64];
+          tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+          tmem_wait_ld();
+          reset_s(tS, magic);                             // reset S for QK_i(t+1)
+          const bool last = (t == nK - 1);
+          float mn;
+          float2 a2, nb2;
+          if constexpr (KMODE == 0) {
+            // A = (q_scale * k_scale) * c; tile max of S*A from the max of S (A > 0)
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (j >= last_valid) x[j] = -INFINITY;     // masked key: p = 2^-inf = 0
+            }
+            // four independent chains over 16 values each: 7 three-input maxima + 1
+            float mq[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              mq[q] = fmaxf(x[16 * q], x[16 * q + 15]);
+#pragma unroll
+              for (int j = 1; j < 15; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
+            }
+            const float xmax = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
+            }
+            const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
+            a2 = make_float2(a, a);
+            nb2 = make_float2(-mn, -mn);
+          } else {
+            // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
+            // fma(S_j, A_j, -mn).  The warp stages the tile's 64 scales in shared
+            // memory (two per lane, one load each) and every thread keeps A_j.
+            const int nv = last ? last_valid : BN;
+            float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
+            kss[2 * lane] = kpair.x;                      // this tile's scales, fetched a tile ago
+            kss[2 * lane + 1] = kpair.y;
+            __syncwarp();
+            // (every lane reads the same address: a broadcast, no bank conflict)
+            float smx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+              const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
+              const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                x[j + u] = __fsub_rn(x[j + u], kMagic);
+                if (j + u < nv) smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c)));
+              }
+            }
+            mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+              const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
+              const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                x[j + u] = (j + u < nv)
+                               ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c), -mn)
+                               : -INFINITY;
+            }
+            __syncwarp();                                   // kss is rewritten next tile
+            a2 = make_float2(1.0f, 1.0f);
+            nb2 = make_float2(0.0f, 0.0f);
+          }
+          tmem_wait_st();                                 // the reset of S has landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + wg);
+          const float old = ex2_approx(__fsub_rn(m, mn));
+          exp_block<0, 64>(x, a2, nb2);
+          // denominator: unquantized probabilities, four independent pair sums
+          float2 acc[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
+#pragma unroll
+          for (int j = 8; j < 64; j += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
+          }
+          acc[0] = fadd2(acc[0], acc[1]);
+          acc[2] = fadd2(acc[2], acc[3]);
+          acc[0] = fadd2(acc[0], acc[2]);
+          den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+          if (t >= 1) {
+            // PV_i(t-1) was issued when this warpgroup finished tile t-1 and has long
+            // completed.  Its completion frees P buffer (t & 1), last read by
+            // PV_i(t-2), and lets this warp rescale its rows of O_i by old before
+            // PV_i(t) accumulates (only if one of its 32 rows' maximum moved).
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((t - 1) & 1), ((t - 1) >> 1) & 1,
+                                                   abort, p.dev_err, kErrTimeoutO));
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D>(tO, old);
+          }
+          tmem_st16(tP + (t & 1) * (BN / 4), pk);
+          tmem_wait_st();                                 // P and any O rescale have landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + 2 * wg + (t & 1));
+          m = mn;
+        }
+        // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization")
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * wg + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
+                                                 abort, p.dev_err, kErrTimeoutO));
+        if (ok) {
+          tc_fence_after();
+          const float inv = rcp_approx(den);
+          const int n = qt * BM + row;
+          const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
+          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_wait_ld();
+            if (n < p.Nq) {
+              uint32_t w[16];
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                             make_float2(inv, inv)),
+                                       make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+              }
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+              d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+              d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            }
           }
         }
       }

@@ -315,7 +315,7 @@ def run_gpu(args):
         step()
         out_host.copy_(pipe.out, non_blocking=True)
 
-    e2e_ms = float("nan")
+    e2e_ms = None
     if not args.no_e2e:
         for _ in range(max(1, args.warmup)):
             e2e_step()
@@ -358,10 +358,11 @@ def run_gpu(args):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "traffic": ATTN_TRAFFIC_BYTES if args.config == "canonical" else None,
-                         "kernel": "attn_fwd_kernel<128,2>",
+                         "kernel": "attn_fwd_kernel<%d,%d,%d>" % (w.D, 2 if w.D <= 128 else 1,
+                                                                  1 if w.hadamard else 0),
                          "peak_source": peak_src,
                          "algorithmic_work": "4*B*H*N^2*D = %.4e ops per launch" % flops},
-            "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12,
+            "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12 if e2e_ms else None,
                     "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": host_qkv.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2},

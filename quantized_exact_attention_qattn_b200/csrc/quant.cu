@@ -180,24 +180,35 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
                                             float* red) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int CH = ROWS * CPR / 128;       // chunks per thread
-  float x[CH][8];
-  float amax = 0.0f;
+  // The raw BF16 chunks stay in registers (4 per chunk) and are unpacked twice,
+  // for the maximum and for the codes, with the same arithmetic both times.
+  uint4 raw[CH];
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
     const int id = threadIdx.x + c * 128;
     const int r = id / CPR, d0 = (id - r * CPR) * 8;
     const int n = row0 + r;
-    if (n < N) {
-      unpack8(*reinterpret_cast<const uint4*>(row_ptr(src, b, n, h) + d0), x[c]);
-      if (mean != nullptr) {
+    raw[c] = (n < N) ? *reinterpret_cast<const uint4*>(row_ptr(src, b, n, h) + d0)
+                     : make_uint4(0, 0, 0, 0);
+  }
+  auto values = [&](int c, float (&x)[8]) {
+    const int id = threadIdx.x + c * 128;
+    const int d0 = (id % CPR) * 8;
+    unpack8(raw[c], x);
+    if (mean != nullptr) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[c][e] = __fsub_rn(x[c][e], mean[d0 + e]);
-      }
+      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], mean[d0 + e]);
+    }
+  };
+  float amax = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[c][e]));
-    } else {
+  for (int c = 0; c < CH; ++c) {
+    const int id = threadIdx.x + c * 128;
+    if (row0 + id / CPR < N) {               // rows past the end take no part
+      float x[8];
+      values(c, x);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[c][e] = 0.0f;
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
     }
   }
   amax = fmaxf(1e-7f, block_max<128>(amax, red));
@@ -209,9 +220,11 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
     const int r = id / CPR, d0 = (id - r * CPR) * 8;
     const int n = row0 + r;
     if (n < N) {
+      float x[8];
+      values(c, x);
       int8_t q[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) q[e] = q8_of(__fmul_rn(x[c][e], f));
+      for (int e = 0; e < 8; ++e) q[e] = q8_of(__fmul_rn(x[e], f));
       uint2 o;
       o.x = pack4_s8(q[0], q[1], q[2], q[3]);
       o.y = pack4_s8(q[4], q[5], q[6], q[7]);
@@ -246,24 +259,40 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
     const int j = blk % a.nK, bh = blk / a.nK;
     const int h = bh % a.Hkv, b = bh / a.Hkv;
     const float* fac = a.vfac + static_cast<int64_t>(bh) * D;
-    constexpr int CPR = D / 8;
-    for (int id = threadIdx.x; id < kKvRows * CPR; id += 128) {
-      const int r = id / CPR, d0 = (id - r * CPR) * 8;
-      const int n = j * kKvRows + r;
-      float x[8];
-      if (n < a.Nkv) {
-        unpack8(*reinterpret_cast<const uint4*>(row_ptr(a.v, b, n, h) + d0), x);
+    // Thread (rg, dc) converts rows 4rg..4rg+3 x dims 8dc..8dc+7 of each 64-dim
+    // slab and writes, per dim, the four rows' codes as one 32-bit word of the
+    // dim-major tile (byte k = row 4rg+k).
+    const int rg = threadIdx.x & 15, dc = threadIdx.x >> 4;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = __fmul_rn(x[e], fac[d0 + e]);
-      } else {
+    for (int slab = 0; slab < D; slab += 64) {
+      const int d0 = slab + 8 * dc;
+      uint4 raw[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+      for (int k = 0; k < 4; ++k) {
+        const int n = j * kKvRows + 4 * rg + k;
+        raw[k] = (n < a.Nkv) ? *reinterpret_cast<const uint4*>(row_ptr(a.v, b, n, h) + d0)
+                             : make_uint4(0, 0, 0, 0);   // zero rows past the end
       }
+      float fv[8];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const uint16_t p = cvt_e4m3x2(x[e], x[e + 1]);
-        tile[(d0 + e) * kKvRows + r] = static_cast<uint8_t>(p & 0xFF);
-        tile[(d0 + e + 1) * kKvRows + r] = static_cast<uint8_t>(p >> 8);
+      for (int e = 0; e < 8; ++e) fv[e] = fac[d0 + e];
+      uint32_t hw[4][4];                                  // [row][dim pair] e4m3 pairs
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float x[8];
+        unpack8(raw[k], x);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2)
+          hw[k][e / 2] = cvt_e4m3x2(__fmul_rn(x[e], fv[e]), __fmul_rn(x[e + 1], fv[e + 1]));
+      }
+      uint32_t* tw = reinterpret_cast<uint32_t*>(tile);
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        const uint32_t u01 = hw[0][e2] | (hw[1][e2] << 16);   // bytes: r0 d, r0 d+1, r1 d, r1 d+1
+        const uint32_t u23 = hw[2][e2] | (hw[3][e2] << 16);
+        const int d = d0 + 2 * e2;
+        tw[(d * kKvRows) / 4 + rg] = __byte_perm(u01, u23, 0x6420);        // dim d, rows 0..3
+        tw[((d + 1) * kKvRows) / 4 + rg] = __byte_perm(u01, u23, 0x7531);  // dim d+1
       }
     }
     __syncthreads();

@@ -192,6 +192,18 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  * a timed-out wait -> QATTN_ERR_TIMEOUT; a CUDA error -> QATTN_ERR_CUDA. */
 qattn_status qattn_check(const int* dev_err, void* stream);
 
+/* ---------------------------------------------------------------- test hook
+ * Failure-path test of the bounded waits (the pages have no counterpart).  After
+ * this call, every qattn_fwd launch in the process skips the K/V copy of key tile
+ * `kv_tile` (0-based, 64 keys each): the tensor-core and softmax waits on that
+ * tile give up after about one second, every role drains its in-flight copies and
+ * MMAs, the kernel returns, and qattn_check reports QATTN_ERR_TIMEOUT with the
+ * error bits set.  The output of such a call is undefined; the CUDA context stays
+ * usable.  kv_tile = -1 (the initial state) turns the hook off.  Process-wide and
+ * not synchronized with launches in flight: for tests only.
+ * Errors: SHAPE if kv_tile < -1. */
+qattn_status qattn_debug_stall_kv_tile(int kv_tile);
+
 /* Human-readable reason of the last non-OK status returned on this thread. */
 const char* qattn_last_error(void);
 

@@ -9,14 +9,15 @@ from __future__ import annotations
 
 import math
 
-from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_check, qattn_fwd, qattn_prep,  # noqa: F401
-                   qattn_quant, qattn_quant_hadamard, qattn_quant_noalloc,
-                   qattn_quant_workspace_bytes, qattn_scores, qattn_version)
+from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_check,  # noqa: F401
+                   qattn_debug_stall_kv_tile, qattn_fwd, qattn_prep, qattn_quant,
+                   qattn_quant_hadamard, qattn_quant_noalloc, qattn_quant_workspace_bytes,
+                   qattn_scores, qattn_version)
 
 __all__ = ["Pipeline", "QAttnError", "qattn_prep", "qattn_quant", "qattn_quant_noalloc",
            "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
-           "qattn_version", "load"]
+           "qattn_debug_stall_kv_tile", "qattn_version", "load"]
 
 
 def _cdiv(a, b):

@@ -21,7 +21,8 @@ QATTN_STATUS = {0: "QATTN_OK", 1: "QATTN_ERR_NULL", 2: "QATTN_ERR_SHAPE", 3: "QA
 
 EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_noalloc",
             "qattn_quant_hadamard",
-            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_last_error", "qattn_version")
+            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_debug_stall_kv_tile",
+            "qattn_last_error", "qattn_version")
 
 
 class QAttnError(RuntimeError):
@@ -62,10 +63,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_fwd.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, vp, vp]
     lib.qattn_scores.argtypes = [i, i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
     lib.qattn_check.argtypes = [vp, vp]
+    lib.qattn_debug_stall_kv_tile.argtypes = [i]
     lib.qattn_last_error.restype = ctypes.c_char_p
     lib.qattn_version.restype = ctypes.c_char_p
     for name in ("qattn_prep", "qattn_quant", "qattn_quant_noalloc", "qattn_quant_hadamard", "qattn_fwd",
-                 "qattn_scores", "qattn_check"):
+                 "qattn_scores", "qattn_check", "qattn_debug_stall_kv_tile"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -147,6 +149,11 @@ def qattn_scores(B, Nq, Nkv, Hq, Hkv, D, q8, k8, tiles, n_tiles, s_out, dev_err,
 
 def qattn_check(dev_err, stream=None):
     _check(load().qattn_check(_ptr(dev_err), _stream(stream)))
+
+
+def qattn_debug_stall_kv_tile(kv_tile: int):
+    """Test hook: later qattn_fwd launches skip the K/V copy of `kv_tile` (-1: off)."""
+    _check(load().qattn_debug_stall_kv_tile(int(kv_tile)))
 
 
 def qattn_version() -> str:

@@ -32,6 +32,7 @@
 #include <cuda_fp16.h>
 
 #include <cmath>
+#include <atomic>
 #include <mutex>
 
 #include "qattn_device.cuh"
@@ -39,6 +40,9 @@
 
 namespace qattn {
 namespace {
+
+// Test hook (qattn_debug_stall_kv_tile): read at each attention launch.
+std::atomic<int> g_stall_tile{-1};
 
 constexpr int BM = 128;   // query rows per tile (TMEM lanes)
 constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
@@ -94,6 +98,7 @@ struct FwdParams {
   int* dev_err;
   int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups;
   float c;
+  int stall_tile;   // test hook: K/V tile whose copy is never issued (-1: none)
 };
 
 // ---------------------------------------------------------------- exp2
@@ -270,6 +275,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (t >= C::STAGES &&
             !mbar_wait(kv_empty + s, ((t / C::STAGES) - 1) & 1, abort, p.dev_err, kErrTimeoutKV))
           break;
+        if (t == p.stall_tile) {   // test hook: this stage's waiters time out
+          issued = t + 1;
+          continue;
+        }
         mbar_arrive_expect_tx(kv_full + s, static_cast<uint32_t>(C::K_BYTES + C::V_BYTES));
         for (int ch = 0; ch < C::NCH; ++ch)
           tma_load_3d(smem + C::SMEM_K + s * C::K_BYTES + ch * (BN * C::KCH), &tmK, kv_full + s,
@@ -280,8 +289,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int dummy = 0;      // drain: every issued copy must land before the CTA may exit
       mbar_wait(q_full, 0, &dummy, p.dev_err, kErrTimeoutDrain);
       for (int u = max(0, issued - C::STAGES); u < issued; ++u)
-        mbar_wait(kv_full + (u % C::STAGES), (u / C::STAGES) & 1, &dummy, p.dev_err,
-                  kErrTimeoutDrain);
+        if (u != p.stall_tile)
+          mbar_wait(kv_full + (u % C::STAGES), (u / C::STAGES) & 1, &dummy, p.dev_err,
+                    kErrTimeoutDrain);
     }
   } else if (warp <= NQT) {
     // ================================================================ MMA issuers
@@ -912,6 +922,7 @@ cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* 
   p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
   p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
   p.c = c;
+  p.stall_tile = g_stall_tile.load();
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) owns an SM
   const int smem = (Cf::SMEM_BYTES + 1024 > 116 * 1024) ? Cf::SMEM_BYTES + 1024 : 116 * 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT, KMODE>,
@@ -956,6 +967,8 @@ cudaError_t launch_scores_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_
 }
 
 }  // namespace
+
+void set_stall_tile(int tile) { g_stall_tile.store(tile); }
 
 cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
                        const float* q_scale, const int8_t* k8, const void* k_scale,

@@ -14,6 +14,13 @@
 
 #include "qattn_internal.h"
 
+#ifndef QATTN_PREP_TOKENS
+#define QATTN_PREP_TOKENS 8
+#endif
+#ifndef QATTN_PREP_PASSES
+#define QATTN_PREP_PASSES 2
+#endif
+
 namespace qattn {
 namespace {
 
@@ -52,13 +59,13 @@ template <int D>
 __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   constexpr int L = D / 8;     // lanes holding one head row
   constexpr int HPW = 32 / L;  // head rows per warp
-  constexpr int MAXP = 8;      // head-row passes whose loads are issued together
-  __shared__ float s_cos[D / 2];
-  __shared__ float s_sin[D / 2];
+  __shared__ float s_cos[QATTN_PREP_TOKENS][D / 2];
+  __shared__ float s_sin[QATTN_PREP_TOKENS][D / 2];
 
-  const int bn = blockIdx.x;
-  const int b = bn / a.N;
-  const int n = bn - b * a.N;
+  const int tiles = (a.N + QATTN_PREP_TOKENS - 1) / QATTN_PREP_TOKENS;
+  const int b = blockIdx.x / tiles;
+  const int n0 = (blockIdx.x - b * tiles) * QATTN_PREP_TOKENS;
+  const int nt = min(QATTN_PREP_TOKENS, a.N - n0);    // tokens of this CTA
   const int half = a.rotary_dim / 2;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -69,105 +76,112 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   const int rot_lanes = a.rotary_dim / 8;
   const int half_lanes = half / 8;
 
-  auto row_src = [&](int hh) {
+  auto row_src = [&](int n, int hh) {
     const bool isq = hh < a.Hq;
     const BNHD src = isq ? a.q : a.k;
     const int h = isq ? hh : hh - a.Hq;
     return src.ptr + b * src.sb + static_cast<int64_t>(n) * src.sn +
            static_cast<int64_t>(h) * src.sh + 8 * l;
   };
-
-  for (int base0 = 0; base0 < total; base0 += MAXP * slots) {
-    // All of this token's row chunks are requested before anything waits on them
-    // (the first time, before the FP64 RoPE table below is computed).
-    uint4 raw[MAXP];
+  constexpr int MAXP = QATTN_PREP_PASSES;   // head-row passes whose loads are issued together
+  uint4 raw[MAXP];
+  auto load_passes = [&](int n, int base0) {
 #pragma unroll
     for (int pidx = 0; pidx < MAXP; ++pidx) {
       const int hh = base0 + pidx * slots + warp * HPW + sub;
       raw[pidx] = make_uint4(0, 0, 0, 0);
-      if (hh < total) raw[pidx] = *reinterpret_cast<const uint4*>(row_src(hh));
+      if (hh < total) raw[pidx] = *reinterpret_cast<const uint4*>(row_src(n, hh));
     }
-    if (base0 == 0) {
-      for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const double inv_freq = pow(a.theta, -(2.0 * i) / static_cast<double>(a.rotary_dim));
-        const double ang = static_cast<double>(a.pos_offset + n) * inv_freq;
-        double sv, cv;
-        sincos(ang, &sv, &cv);
-        s_cos[i] = bf16_round_f64(cv);
-        s_sin[i] = bf16_round_f64(sv);
-      }
-      __syncthreads();
-    }
+  };
 
-#pragma unroll
-    for (int pidx = 0; pidx < MAXP; ++pidx) {
-      const int base = base0 + pidx * slots;
-      if (base >= total) break;                   // uniform over the CTA
-      const int hh = base + warp * HPW + sub;
-      const bool valid = hh < total;
-      const bool isq = hh < a.Hq;
-      const int h = isq ? hh : hh - a.Hq;
-      const uint16_t* w = isq ? a.qw : a.kw;
-      float x[8];
-      x[0] = bf16_lo(raw[pidx].x); x[1] = bf16_hi(raw[pidx].x);
-      x[2] = bf16_lo(raw[pidx].y); x[3] = bf16_hi(raw[pidx].y);
-      x[4] = bf16_lo(raw[pidx].z); x[5] = bf16_hi(raw[pidx].z);
-      x[6] = bf16_lo(raw[pidx].w); x[7] = bf16_hi(raw[pidx].w);
+  // The first loads go out before the FP64 RoPE tables of all the CTA's tokens
+  // are computed (by all threads at once), so the table latency overlaps them.
+  load_passes(n0, 0);
+  for (int idx = threadIdx.x; idx < nt * half; idx += blockDim.x) {
+    const int k = idx / half, i = idx - k * half;
+    const double inv_freq = pow(a.theta, -(2.0 * i) / static_cast<double>(a.rotary_dim));
+    const double ang = static_cast<double>(a.pos_offset + n0 + k) * inv_freq;
+    double sv, cv;
+    sincos(ang, &sv, &cv);
+    s_cos[k][i] = bf16_round_f64(cv);
+    s_sin[k][i] = bf16_round_f64(sv);
+  }
+  __syncthreads();
 
-      // ---- RMSNorm (skipped when this tensor has no weight; uniform per warp
-      //      only when Hq and Hkv rows do not share a warp, so every lane takes
-      //      part in the shuffles regardless)
-      float ss = __fmul_rn(x[0], x[0]);
+  for (int k = 0; k < nt; ++k) {
+    const int n = n0 + k;
+    for (int base0 = 0; base0 < total; base0 += MAXP * slots) {
+      if (k > 0 || base0 > 0) load_passes(n, base0);
 #pragma unroll
-      for (int e = 1; e < 8; ++e) ss = __fadd_rn(ss, __fmul_rn(x[e], x[e]));
-#pragma unroll
-      for (int off = L / 2; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-      float y[8];
-      if (w != nullptr) {
-        const float ms = __fmul_rn(ss, 1.0f / D);
-        const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
-        const uint4 wr = *reinterpret_cast<const uint4*>(w + 8 * l);
-        const float wv[8] = {bf16_lo(wr.x), bf16_hi(wr.x), bf16_lo(wr.y), bf16_hi(wr.y),
-                             bf16_lo(wr.z), bf16_hi(wr.z), bf16_lo(wr.w), bf16_hi(wr.w)};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = bf16_rn(__fmul_rn(bf16_rn(__fmul_rn(x[e], r)), wv[e]));
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = x[e];
-      }
+      for (int pidx = 0; pidx < MAXP; ++pidx) {
+        const int base = base0 + pidx * slots;
+        if (base >= total) break;                   // uniform over the CTA
+        const int hh = base + warp * HPW + sub;
+        const bool valid = hh < total;
+        const bool isq = hh < a.Hq;
+        const int h = isq ? hh : hh - a.Hq;
+        const uint16_t* w = isq ? a.qw : a.kw;
+        float x[8];
+        x[0] = bf16_lo(raw[pidx].x); x[1] = bf16_hi(raw[pidx].x);
+        x[2] = bf16_lo(raw[pidx].y); x[3] = bf16_hi(raw[pidx].y);
+        x[4] = bf16_lo(raw[pidx].z); x[5] = bf16_hi(raw[pidx].z);
+        x[6] = bf16_lo(raw[pidx].w); x[7] = bf16_hi(raw[pidx].w);
 
-      // ---- split-half RoPE: lane l < R/16 pairs with lane l + R/16
-      if (rot_lanes > 0) {
-        const int pl = (l < half_lanes) ? l + half_lanes : (l < rot_lanes ? l - half_lanes : l);
-        const int src_lane = sub * L + pl;
-        float o[8];
+        // ---- RMSNorm (skipped when this tensor has no weight; uniform per warp
+        //      only when Hq and Hkv rows do not share a warp, so every lane takes
+        //      part in the shuffles regardless)
+        float ss = __fmul_rn(x[0], x[0]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = __shfl_sync(0xffffffffu, y[e], src_lane);
-        if (l < half_lanes) {
+        for (int e = 1; e < 8; ++e) ss = __fadd_rn(ss, __fmul_rn(x[e], x[e]));
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = 8 * l + e;
-            y[e] = bf16_rn(__fsub_rn(__fmul_rn(y[e], s_cos[i]), __fmul_rn(o[e], s_sin[i])));
-          }
-        } else if (l < rot_lanes) {
+        for (int off = L / 2; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+        float y[8];
+        if (w != nullptr) {
+          const float ms = __fmul_rn(ss, 1.0f / D);
+          const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
+          const uint4 wr = *reinterpret_cast<const uint4*>(w + 8 * l);
+          const float wv[8] = {bf16_lo(wr.x), bf16_hi(wr.x), bf16_lo(wr.y), bf16_hi(wr.y),
+                               bf16_lo(wr.z), bf16_hi(wr.z), bf16_lo(wr.w), bf16_hi(wr.w)};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = 8 * l + e - half;
-            y[e] = bf16_rn(__fadd_rn(__fmul_rn(y[e], s_cos[i]), __fmul_rn(o[e], s_sin[i])));
+          for (int e = 0; e < 8; ++e) y[e] = bf16_rn(__fmul_rn(bf16_rn(__fmul_rn(x[e], r)), wv[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = x[e];
+        }
+
+        // ---- split-half RoPE: lane l < R/16 pairs with lane l + R/16
+        if (rot_lanes > 0) {
+          const int pl = (l < half_lanes) ? l + half_lanes : (l < rot_lanes ? l - half_lanes : l);
+          const int src_lane = sub * L + pl;
+          float o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = __shfl_sync(0xffffffffu, y[e], src_lane);
+          if (l < half_lanes) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int i = 8 * l + e;
+              y[e] = bf16_rn(__fsub_rn(__fmul_rn(y[e], s_cos[k][i]), __fmul_rn(o[e], s_sin[k][i])));
+            }
+          } else if (l < rot_lanes) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int i = 8 * l + e - half;
+              y[e] = bf16_rn(__fadd_rn(__fmul_rn(y[e], s_cos[k][i]), __fmul_rn(o[e], s_sin[k][i])));
+            }
           }
         }
-      }
 
-      if (valid) {
-        const int H = isq ? a.Hq : a.Hkv;
-        uint16_t* dst = (isq ? a.q_out : a.k_out) +
-                        ((static_cast<int64_t>(b) * a.N + n) * H + h) * D + 8 * l;
-        uint4 o;
-        o.x = bf16_bits(y[0]) | (bf16_bits(y[1]) << 16);
-        o.y = bf16_bits(y[2]) | (bf16_bits(y[3]) << 16);
-        o.z = bf16_bits(y[4]) | (bf16_bits(y[5]) << 16);
-        o.w = bf16_bits(y[6]) | (bf16_bits(y[7]) << 16);
-        *reinterpret_cast<uint4*>(dst) = o;
+        if (valid) {
+          const int H = isq ? a.Hq : a.Hkv;
+          uint16_t* dst = (isq ? a.q_out : a.k_out) +
+                          ((static_cast<int64_t>(b) * a.N + n) * H + h) * D + 8 * l;
+          uint4 o;
+          o.x = bf16_bits(y[0]) | (bf16_bits(y[1]) << 16);
+          o.y = bf16_bits(y[2]) | (bf16_bits(y[3]) << 16);
+          o.z = bf16_bits(y[4]) | (bf16_bits(y[5]) << 16);
+          o.w = bf16_bits(y[6]) | (bf16_bits(y[7]) << 16);
+          *reinterpret_cast<uint4*>(dst) = o;
+        }
       }
     }
   }
@@ -180,7 +194,8 @@ cudaError_t launch_prep(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD k,
                         double theta, int64_t pos_offset, uint16_t* q_out, uint16_t* k_out,
                         cudaStream_t st) {
   PrepArgs a{q, k, qw, kw, q_out, k_out, B, N, Hq, Hkv, rotary_dim, eps, theta, pos_offset};
-  const dim3 grid(static_cast<unsigned>(B) * static_cast<unsigned>(N));
+  const dim3 grid(static_cast<unsigned>(B) *
+                  static_cast<unsigned>((N + QATTN_PREP_TOKENS - 1) / QATTN_PREP_TOKENS));
   switch (D) {
     case 64: prep_kernel<64><<<grid, 256, 0, st>>>(a); break;
     case 128: prep_kernel<128><<<grid, 256, 0, st>>>(a); break;

@@ -226,6 +226,12 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const 
   return QATTN_OK;
 }
 
+qattn_status qattn_debug_stall_kv_tile(int kv_tile) {
+  if (kv_tile < -1) return fail(QATTN_ERR_SHAPE, "debug_stall_kv_tile: tile must be >= -1");
+  qattn::set_stall_tile(kv_tile);
+  return QATTN_OK;
+}
+
 qattn_status qattn_check(const int* dev_err, void* stream) {
   if (dev_err == nullptr) return fail(QATTN_ERR_NULL, "check: null dev_err");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -47,6 +47,9 @@ cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                   uint8_t* v8t, cudaStream_t st);
 
 // attn_fwd.cu
+// Test hook: K/V tile whose copy later attention launches skip (-1: none).
+void set_stall_tile(int tile);
+
 cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
                        const float* q_scale, const int8_t* k8, const void* k_scale,
                        int k_scale_mode, const uint8_t* v8t, const float* v_scale,

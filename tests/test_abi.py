@@ -117,3 +117,9 @@ def test_scores_refusals(lib):
     assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) == 2
     assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, None, 4, FAKE, FAKE, None) == 1
     assert lib.qattn_check(None, None) == 1
+
+
+def test_stall_hook_refuses_negative_tiles_and_resets(lib):
+    assert lib.qattn_debug_stall_kv_tile(-2) == 2          # QATTN_ERR_SHAPE
+    assert "kv_tile" in lib.qattn_last_error().decode() or "tile" in lib.qattn_last_error().decode()
+    assert lib.qattn_debug_stall_kv_tile(-1) == 0          # off (the initial state)

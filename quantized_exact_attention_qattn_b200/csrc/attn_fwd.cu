@@ -35,20 +35,18 @@
 #include <atomic>
 #include <mutex>
 
-#include "qattn_device.cuh"
-#include "qattn_internal.h"
+#include "attn_common.cuh"
 
 namespace qattn {
-namespace {
 
 // Test hook (qattn_debug_stall_kv_tile): read at each attention launch.
-std::atomic<int> g_stall_tile{-1};
+static std::atomic<int> g_stall_tile{-1};
+int stall_tile() { return g_stall_tile.load(); }
 
-constexpr int BM = 128;   // query rows per tile (TMEM lanes)
+namespace {
+using namespace attn;
+
 constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
-constexpr float kMInit = -5000000.0f;
-constexpr float kFp8Offset = 8.807f;
-constexpr float kMasked = -5000000.0f;
 
 template <int D, int NQT>
 struct Cfg {
@@ -89,101 +87,6 @@ struct Cfg {
   static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
   static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
 };
-
-struct FwdParams {
-  const float* q_scale;
-  const void* k_scale;
-  const float* v_scale;
-  uint16_t* out;
-  int* dev_err;
-  int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups;
-  float c;
-  int stall_tile;   // test hook: K/V tile whose copy is never issued (-1: none)
-};
-
-// ---------------------------------------------------------------- exp2
-// Columns j with (j % 8) < kPolyPer8 evaluate 2^t with an FMA-pipe polynomial,
-// the rest with the MUFU ex2.approx, so both pipes share the exponentials.
-#ifndef QATTN_POLY_PER8
-#define QATTN_POLY_PER8 2
-#endif
-constexpr int kPolyPer8 = QATTN_POLY_PER8;
-constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: x + kMagic rounds x to an integer
-// 2^f on [-1/2, 1/2], degree 5, relative minimax (fit_exp2.py), max relative error
-// 2.3e-7 in FP32: about that of ex2.approx, so both paths round P to E4M3 alike.
-constexpr float kC0 = 1.000000119e+00f, kC1 = 6.931469440e-01f, kC2 = 2.402212024e-01f,
-                kC3 = 5.550713092e-02f, kC4 = 9.675540961e-03f, kC5 = 1.327647245e-03f;
-
-// 2^t for two values at once: n = round(t), f = t - n, 2^t = poly(f) * 2^n with
-// n added to the exponent field.  t is clamped at -126 so that the exponent of
-// the result stays >= 0 (a tiny or subnormal positive value, never a wrap).
-__device__ __forceinline__ float2 exp2_poly2(float2 t) {
-  t.x = fmaxf(t.x, -126.0f);
-  t.y = fmaxf(t.y, -126.0f);
-  const float2 j = fadd2(t, make_float2(kMagic, kMagic));          // round to integer
-  const float2 n = fadd2(j, make_float2(-kMagic, -kMagic));        // exact
-  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), t);         // t - n, exact
-  float2 q = ffma2(make_float2(kC5, kC5), f, make_float2(kC4, kC4));
-  q = ffma2(q, f, make_float2(kC3, kC3));
-  q = ffma2(q, f, make_float2(kC2, kC2));
-  q = ffma2(q, f, make_float2(kC1, kC1));
-  q = ffma2(q, f, make_float2(kC0, kC0));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
-}
-
-template <int J>
-__device__ __forceinline__ float2 exp2_pair(float2 t) {
-  if constexpr ((J % 8) < kPolyPer8) {
-    return exp2_poly2(t);
-  } else {
-    return make_float2(ex2_approx(t.x), ex2_approx(t.y));
-  }
-}
-
-// x[j] holds the exact FP32 score S_j; the exponent is fma(S_j, A, -mn).  Columns
-// J .. END-1 of the row's N values, two at a time.
-template <int J, int END, int N>
-__device__ __forceinline__ void exp_block(float (&x)[N], float2 a2, float2 nb2) {
-  if constexpr (J < END) {
-    const float2 t = ffma2(make_float2(x[J], x[J + 1]), a2, nb2);
-    const float2 e = exp2_pair<J>(t);
-    x[J] = e.x;
-    x[J + 1] = e.y;
-    exp_block<J + 2, END>(x, a2, nb2);
-  }
-}
-
-// S <- kMagic bits for this warp's 32 rows, 64 columns (four 16-column stores).
-__device__ __forceinline__ void reset_s(uint32_t tS, const uint32_t (&m)[16]) {
-#pragma unroll
-  for (int c = 0; c < 64; c += 16) tmem_st16(tS + c, m);
-}
-
-// O <- O * o for this warp's 32 rows and NCOL columns of O (tensor memory), 64
-// (or, for a 32-column block, 32) columns at a time.
-template <int NCOL>
-__device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
-  constexpr int CH = (NCOL % 64 == 0) ? 64 : 32;
-#pragma unroll 1
-  for (int c0 = 0; c0 < NCOL; c0 += CH) {
-    uint32_t r[CH];
-#pragma unroll
-    for (int c = 0; c < CH; c += 32)
-      tmem_ld32(tO + c0 + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < CH; j += 2) {
-      const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
-                             make_float2(o, o));
-      r[j] = __float_as_uint(v.x);
-      r[j + 1] = __float_as_uint(v.y);
-    }
-#pragma unroll
-    for (int c = 0; c < CH; c += 32)
-      tmem_st32(tO + c0 + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
-  }
-}
 
 template <int D, int NQT, int KMODE>
 __global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
@@ -866,39 +769,6 @@ scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// 3-D uint8 tensor map: dims {inner, rows, planes}, row pitch = inner bytes.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
-              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {inner, rows, planes};
-  const cuuint64_t strides[2] = {inner, inner * rows};
-  const cuuint32_t box[3] = {box_inner, box_rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int NQT, int KMODE>
 cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
                          const float* q_scale, const int8_t* k8, const void* k_scale,
@@ -922,7 +792,7 @@ cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* 
   p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
   p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
   p.c = c;
-  p.stall_tile = g_stall_tile.load();
+  p.stall_tile = stall_tile();
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) owns an SM
   const int smem = (Cf::SMEM_BYTES + 1024 > 116 * 1024) ? Cf::SMEM_BYTES + 1024 : 116 * 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT, KMODE>,

@@ -12,6 +12,7 @@
 // while the token's row loads are already in flight.
 #include <cuda_bf16.h>
 
+#include "qattn_device.cuh"
 #include "qattn_internal.h"
 
 #ifndef QATTN_PREP_TOKENS
@@ -50,17 +51,21 @@ __device__ __forceinline__ float bf16_round_f64(double x) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t bf16_bits(float f) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+// Two FP32 values -> one BF16 pair (x in the low half), each rounded to nearest even.
+__device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
-__device__ __forceinline__ float bf16_rn(float f) { return __uint_as_float(bf16_bits(f) << 16); }
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   constexpr int L = D / 8;     // lanes holding one head row
   constexpr int HPW = 32 / L;  // head rows per warp
-  __shared__ float s_cos[QATTN_PREP_TOKENS][D / 2];
-  __shared__ float s_sin[QATTN_PREP_TOKENS][D / 2];
+  __shared__ __align__(16) float s_cos[QATTN_PREP_TOKENS][D / 2];
+  __shared__ __align__(16) float s_sin[QATTN_PREP_TOKENS][D / 2];
 
   const int tiles = (a.N + QATTN_PREP_TOKENS - 1) / QATTN_PREP_TOKENS;
   const int b = blockIdx.x / tiles;
@@ -135,38 +140,50 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
         for (int e = 1; e < 8; ++e) ss = __fadd_rn(ss, __fmul_rn(x[e], x[e]));
 #pragma unroll
         for (int off = L / 2; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-        float y[8];
+        // Packed FP32 pairs and BF16 pairs from here on: every element still sees
+        // exactly the same roundings (RN products, RN sums, BF16 RN) as above.
+        uint32_t yb[4];                                  // BF16 pairs, dims 8l + 2j, 8l + 2j + 1
         if (w != nullptr) {
           const float ms = __fmul_rn(ss, 1.0f / D);
           const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
           const uint4 wr = *reinterpret_cast<const uint4*>(w + 8 * l);
-          const float wv[8] = {bf16_lo(wr.x), bf16_hi(wr.x), bf16_lo(wr.y), bf16_hi(wr.y),
-                               bf16_lo(wr.z), bf16_hi(wr.z), bf16_lo(wr.w), bf16_hi(wr.w)};
+          const uint32_t wv[4] = {wr.x, wr.y, wr.z, wr.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = bf16_rn(__fmul_rn(bf16_rn(__fmul_rn(x[e], r)), wv[e]));
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t xr = bf16x2_rn(fmul2(make_float2(x[2 * j], x[2 * j + 1]), make_float2(r, r)));
+            yb[j] = bf16x2_rn(fmul2(unpack_bf16x2(xr), unpack_bf16x2(wv[j])));
+          }
         } else {
+          const uint32_t xv[4] = {raw[pidx].x, raw[pidx].y, raw[pidx].z, raw[pidx].w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = x[e];
+          for (int j = 0; j < 4; ++j) yb[j] = xv[j];
         }
 
-        // ---- split-half RoPE: lane l < R/16 pairs with lane l + R/16
+        // ---- split-half RoPE: lane l < R/16 pairs with lane l + R/16.  Both halves
+        //      as y*cos + o*sv, sv = -sin (first half) or +sin (second half), which
+        //      is bit for bit y*cos - o*sin or y*cos + o*sin; other lanes pass through.
         if (rot_lanes > 0) {
           const int pl = (l < half_lanes) ? l + half_lanes : (l < rot_lanes ? l - half_lanes : l);
           const int src_lane = sub * L + pl;
-          float o[8];
+          uint32_t ob[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[e] = __shfl_sync(0xffffffffu, y[e], src_lane);
-          if (l < half_lanes) {
+          for (int j = 0; j < 4; ++j) ob[j] = __shfl_sync(0xffffffffu, yb[j], src_lane);
+          if (l < rot_lanes) {
+            const bool first = l < half_lanes;
+            const int i0 = first ? 8 * l : 8 * l - half;
+            const float4 c0 = *reinterpret_cast<const float4*>(&s_cos[k][i0]);
+            const float4 c1 = *reinterpret_cast<const float4*>(&s_cos[k][i0 + 4]);
+            const float4 n0 = *reinterpret_cast<const float4*>(&s_sin[k][i0]);
+            const float4 n1 = *reinterpret_cast<const float4*>(&s_sin[k][i0 + 4]);
+            const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const float sn = first ? -1.0f : 1.0f;       // exact sign flip
+            const float sv[8] = {sn * n0.x, sn * n0.y, sn * n0.z, sn * n0.w,
+                                 sn * n1.x, sn * n1.y, sn * n1.z, sn * n1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int i = 8 * l + e;
-              y[e] = bf16_rn(__fsub_rn(__fmul_rn(y[e], s_cos[k][i]), __fmul_rn(o[e], s_sin[k][i])));
-            }
-          } else if (l < rot_lanes) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int i = 8 * l + e - half;
-              y[e] = bf16_rn(__fadd_rn(__fmul_rn(y[e], s_cos[k][i]), __fmul_rn(o[e], s_sin[k][i])));
+            for (int j = 0; j < 4; ++j) {
+              const float2 yc = fmul2(unpack_bf16x2(yb[j]), make_float2(cv[2 * j], cv[2 * j + 1]));
+              const float2 os = fmul2(unpack_bf16x2(ob[j]), make_float2(sv[2 * j], sv[2 * j + 1]));
+              yb[j] = bf16x2_rn(fadd2(yc, os));
             }
           }
         }
@@ -175,12 +192,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
           const int H = isq ? a.Hq : a.Hkv;
           uint16_t* dst = (isq ? a.q_out : a.k_out) +
                           ((static_cast<int64_t>(b) * a.N + n) * H + h) * D + 8 * l;
-          uint4 o;
-          o.x = bf16_bits(y[0]) | (bf16_bits(y[1]) << 16);
-          o.y = bf16_bits(y[2]) | (bf16_bits(y[3]) << 16);
-          o.z = bf16_bits(y[4]) | (bf16_bits(y[5]) << 16);
-          o.w = bf16_bits(y[6]) | (bf16_bits(y[7]) << 16);
-          *reinterpret_cast<uint4*>(dst) = o;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
         }
       }
     }

@@ -49,6 +49,7 @@ cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
 // attn_fwd.cu
 // Test hook: K/V tile whose copy later attention launches skip (-1: none).
 void set_stall_tile(int tile);
+int stall_tile();
 
 cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
                        const float* q_scale, const int8_t* k8, const void* k_scale,

@@ -19,11 +19,15 @@
 //               scores, the online-softmax update, tcgen05.st of its 64 FP8
 //               probabilities, the O rescale of its row (only in warps where some
 //               row's maximum moved, after the previous P.V completed), and the
-//               final normalisation + BF16 store.
+//               final normalisation + BF16 store.  S is preloaded with the bits
+//               of 1.5 * 2^23 and QK accumulates onto them, so the scores read
+//               back as FP32 with one packed subtract per pair and no conversion.
 //   warps 3..   D = 256: two warpgroups per query tile, one per half of the 64
 //               keys (and of the O columns); the two warps on the same rows swap
 //               their half-row maxima through shared memory every tile, and add
-//               their partial denominators at the end.
+//               their partial denominators at the end.  Here QK overwrites S and
+//               the warps convert their 32 INT32 scores with I2F, which frees S
+//               for the next QK right after the load.
 // The two query tiles' chains are independent, so while one warpgroup runs the
 // softmax of its tile the tensor core works for the other.  Every wait is
 // bounded; a timeout sets a device error bit and all roles drain.
@@ -215,7 +219,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint64_t ad = smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          mma_i8_ss(tS, ad, bd, C::IDESC_QK, 1u);   // onto the kMagic bits already in S
+          // split layout: the first K step overwrites S; full rows: onto the kMagic bits
+          mma_i8_ss(tS, ad, bd, C::IDESC_QK, (C::SPLIT && kk == 0) ? 0u : 1u);
         }
         tc_commit(s_full + i);
       };
@@ -287,21 +292,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         };
         float kone_next = 0.0f;
         if constexpr (KMODE == 1) kone_next = load_kone(0);
-        // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
-        // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
-        // conversion is needed.  Each half resets its own 32 columns.
-        uint32_t magic[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) magic[j] = 0x4B400000u;
-        auto reset_own = [&]() {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) tmem_st8(tS_own + c, magic);
-        };
-        reset_own();
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + i);       // s_free phase t: QK_i(t) may accumulate
+        // s_free phase t: QK_i(t) may overwrite S_i (phase 0 needs nothing read)
+        if (lane == 0) mbar_arrive(s_free + i);
         for (int t = 0; ok && t < nK; ++t) {
           const float ks_cur = ks_next;
           if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
@@ -315,7 +307,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float x[32];                                    // this half's 32 scores
           tmem_ld32(tS_own, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
           tmem_wait_ld();
-          reset_own();                                    // reset S for QK_i(t+1)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + i);         // S_i(t) read: QK_i(t+1) may overwrite it
+          // INT32 scores to FP32: exact, |S| <= D * 127^2 < 2^24
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
           const bool last = (t == nK - 1);
           const int nv = last ? last_valid : BN;          // valid keys in this tile
           const int own0 = hf * 32;                       // first key of this half
@@ -356,14 +353,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               ok = false;
               break;
             }
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
-              x[j] = sj.x;
-              x[j + 1] = sj.y;
-            }
             const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            const float smax = __fmul_rn(xmax, a);
             mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
             a2 = make_float2(a, a);
             nb2 = make_float2(-mn, -mn);
@@ -380,11 +371,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               const float4 km = *reinterpret_cast<const float4*>(kss + j);
               const float kkm[4] = {km.x, km.y, km.z, km.w};
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                x[j + u] = __fsub_rn(x[j + u], kMagic);
+              for (int u = 0; u < 4; ++u)
                 if (own0 + j + u < nv)
                   smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kkm[u]), p.c)));
-              }
             }
             mn = fmaxf(m, __fsub_rn(pair_max(smx), kFp8Offset));
             if (!pair_ok) {
@@ -405,10 +394,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             a2 = make_float2(1.0f, 1.0f);
             nb2 = make_float2(0.0f, 0.0f);
           }
-          tmem_wait_st();                                 // the reset of S has landed
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_free + i);
           const float old = ex2_approx(__fsub_rn(m, mn));
           exp_block<0, 32>(x, a2, nb2);
           // partial denominator: unquantized probabilities, four independent pair sums

@@ -28,8 +28,9 @@
 //               their partial denominators at the end.  Here QK overwrites S and
 //               the warps convert their 32 INT32 scores with I2F, which frees S
 //               for the next QK right after the load.
-// The two query tiles' chains are independent, so while one warpgroup runs the
-// softmax of its tile the tensor core works for the other.  Every wait is
+// The query tiles' chains (two per CTA at D = 128, three at D = 64, where the
+// smaller O leaves TMEM room for a third) are independent, so while one warpgroup
+// runs the softmax of its tile the tensor core works for the others.  Every wait is
 // bounded; a timeout sets a device error bit and all roles drain.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -831,8 +832,8 @@ cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int
                        float score_c, uint16_t* out, int* dev_err, cudaStream_t st,
                        const char** why) {
   switch (D) {
-    case 64:
-      return launch_fwd_d<64, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
+    case 64:   // three query tiles: O 192 + S 192 + P 96 of the 512 TMEM columns
+      return launch_fwd_d<64, 3>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
                                  v_scale, score_c, out, dev_err, st, why);
     case 128:
       return launch_fwd_d<128, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,

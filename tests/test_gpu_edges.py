@@ -30,6 +30,7 @@ EDGE = [
     (1, 200, 8, 2, 256, True),
     (1, 729, 2, 2, 64, False),
     (2, 768, 2, 2, 128, True),
+    (1, 500, 2, 2, 128, True),       # four query tiles: a last group of one
     (1, 1000, 6, 3, 128, True),
 ]
 
@@ -72,6 +73,24 @@ def test_hadamard_small(Nq, Nkv, Hq, Hkv, D):
     for key in ("q8", "q_scale", "k8", "k_scale", "v8t", "v_scale"):
         assert np.array_equal(host(getattr(pipe, key)), ref[key]), key
     assert_out_close(host(pipe.out), ref["out"], "hadamard")
+
+
+@pytest.mark.parametrize("Nq,Nkv,Hq,Hkv", [(300, 500, 4, 2), (700, 1000, 2, 1)])
+def test_per_token_k_scales_d128(Nq, Nkv, Hq, Hkv):
+    # qattn_fwd with per-token FP16 K scales at D = 128 (the rotated quantization
+    # of the oracle only serves to produce per-token-scaled inputs here)
+    w = synth.make("gqa_chunk", Nq=Nq, Nkv=Nkv, Hq=Hq, Hkv=Hkv, D=128, seed=Nq + Nkv)
+    q8, qs, k8, ks16, v8t, vs = O.quant_hadamard(w.q, w.k, w.v)
+    out, _, _ = O.attention(q8, qs, k8, ks16, v8t, vs, Nkv, k_scale_mode=1)
+    pipe = qa.Pipeline(1, Nq, Nkv, Hq, Hkv, 128, hadamard=True, device=DEV)
+    for name, arr in (("q8", q8), ("q_scale", qs), ("k8", k8), ("k_scale", ks16.view(np.int16)),
+                      ("v8t", v8t), ("v_scale", vs)):
+        dst = getattr(pipe, name)
+        src = torch.from_numpy(np.ascontiguousarray(arr))
+        dst.copy_(src.view(dst.dtype) if src.dtype.itemsize == dst.dtype.itemsize else src)
+    pipe.run_fwd()
+    pipe.check()
+    assert_out_close(host(pipe.out), out, "per-token K scales, D=128")
 
 
 def test_interleaved_strided_equals_contiguous():

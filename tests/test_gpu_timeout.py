@@ -6,7 +6,8 @@ Each such wait gives up after its bound (about one second), the kernel drains it
 in-flight copies and MMAs and returns, and qattn_check reports QATTN_ERR_TIMEOUT
 with the error bits.  The CUDA context stays usable: the next call, with the hook
 off, gives exactly the output of the call before the failure.  Covered for the
-one-warpgroup softmax (D=128, D=64) and the split one (D=256, per-token scales).
+one-warpgroup softmax (D=128 with pooled S buffers and P in shared memory, D=64)
+and the split one (D=256, per-token scales).
 """
 import pytest
 import torch
@@ -19,7 +20,7 @@ from gpu_helpers import run_pipeline
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name, tile", [("small", 1), ("encoder", 3), ("gqa_chunk", 7)])
+@pytest.mark.parametrize("name, tile", [("small", 1), ("mid", 5), ("encoder", 3), ("gqa_chunk", 7)])
 def test_stalled_copy_times_out_and_the_context_recovers(name, tile):
     w = synth.make(name)
     pipe = run_pipeline(w)                      # a good call first

@@ -366,37 +366,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * 32;
             kss[lane] = kone;                             // this tile's scale, fetched a tile ago
             __syncwarp();
+            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;
+            if (!last) {
+              smx = kt_tile_max<32>(x, kss, qs2, c2);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 km = *reinterpret_cast<const float4*>(kss + j);
-              const float kkm[4] = {km.x, km.y, km.z, km.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                if (own0 + j + u < nv)
-                  smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kkm[u]), p.c)));
+              for (int j = 0; j < 32; ++j)
+                if (own0 + j < nv)
+                  smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[j]), p.c)));
             }
             mn = fmaxf(m, __fsub_rn(pair_max(smx), kFp8Offset));
             if (!pair_ok) {
               ok = false;
               break;
             }
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 km = *reinterpret_cast<const float4*>(kss + j);
-              const float kkm[4] = {km.x, km.y, km.z, km.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                x[j + u] = (own0 + j + u < nv)
-                               ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kkm[u]), p.c), -mn)
-                               : -INFINITY;
-            }
-            __syncwarp();                                   // kss is rewritten next tile
-            a2 = make_float2(1.0f, 1.0f);
-            nb2 = make_float2(0.0f, 0.0f);
+            nb2 = make_float2(-mn, -mn);
           }
           const float old = ex2_approx(__fsub_rn(m, mn));
-          exp_block<0, 32>(x, a2, nb2);
+          if constexpr (KMODE == 0) {
+            exp_block<0, 32>(x, a2, nb2);
+          } else {
+            exp_block_kt<0, 32>(x, ks_stage + (warp - C::SOFTMAX_WARP0) * 32, make_float2(qs, qs),
+                                make_float2(p.c, p.c), nb2);
+            __syncwarp();                                 // kss is rewritten next tile
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (own0 + j >= nv) x[j] = 0.0f;          // masked key: p = 0
+            }
+          }
           // partial denominator: unquantized probabilities, four independent pair sums
           float2 acc[4];
 #pragma unroll
@@ -560,38 +559,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             kss[2 * lane + 1] = kpair.y;
             __syncwarp();
             // (every lane reads the same address: a broadcast, no bank conflict)
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
+            }
+            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;
+            if (!last) {
+              smx = kt_tile_max<64>(x, kss, qs2, c2);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 64; j += 4) {
-              const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
-              const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                x[j + u] = __fsub_rn(x[j + u], kMagic);
-                if (j + u < nv) smx = fmaxf(smx, __fmul_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c)));
-              }
+              for (int j = 0; j < 64; ++j)
+                if (j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[j]), p.c)));
             }
             mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
-#pragma unroll
-            for (int j = 0; j < 64; j += 4) {
-              const float4 k4 = *reinterpret_cast<const float4*>(kss + j);
-              const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                x[j + u] = (j + u < nv)
-                               ? __fmaf_rn(x[j + u], __fmul_rn(__fmul_rn(qs, kk[u]), p.c), -mn)
-                               : -INFINITY;
-            }
-            __syncwarp();                                   // kss is rewritten next tile
-            a2 = make_float2(1.0f, 1.0f);
-            nb2 = make_float2(0.0f, 0.0f);
+            nb2 = make_float2(-mn, -mn);
           }
           tmem_wait_st();                                 // the reset of S has landed
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + wg);
           const float old = ex2_approx(__fsub_rn(m, mn));
-          exp_block<0, 64>(x, a2, nb2);
+          if constexpr (KMODE == 0) {
+            exp_block<0, 64>(x, a2, nb2);
+          } else {
+            exp_block_kt<0, 64>(x, ks_stage + (warp - C::SOFTMAX_WARP0) * BN, make_float2(qs, qs),
+                                make_float2(p.c, p.c), nb2);
+            __syncwarp();                                 // kss is rewritten next tile
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (j >= last_valid) x[j] = 0.0f;         // masked key: p = 0
+            }
+          }
           // denominator: unquantized probabilities, four independent pair sums
           float2 acc[4];
 #pragma unroll

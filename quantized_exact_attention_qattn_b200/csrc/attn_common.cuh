@@ -20,6 +20,7 @@ constexpr float kMInit = -5000000.0f;
 constexpr float kFp8Offset = 8.807f;
 
 struct FwdParams {
+  const int8_t* q8;     // [B,Hq,Nq,D]: read directly when Q lives in tensor memory
   const float* q_scale;
   const void* k_scale;
   const float* v_scale;

@@ -62,8 +62,12 @@ struct Cfg {
   static constexpr int Q_BYTES = BM * D;
   static constexpr int K_BYTES = BN * D;
   static constexpr int V_BYTES = D * BN;
+  // Q in tensor memory (A operand of QK read from TMEM, so each QK MMA reads only
+  // its K tile from shared memory) wherever the columns allow: D = 128 with two
+  // query tiles, D = 256 with one; D = 64 with three keeps Q in shared memory.
+  static constexpr bool Q_TMEM = (D != 64);
   static constexpr int SMEM_Q = 0;
-  static constexpr int SMEM_K = SMEM_Q + NQT * Q_BYTES;
+  static constexpr int SMEM_K = SMEM_Q + (Q_TMEM ? 0 : NQT * Q_BYTES);
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
   // Softmax layout: one warpgroup per query tile owning whole 64-key rows, or (for
   // D = 256, where the longer P.V gives the softmax more time per tile and more
@@ -76,7 +80,7 @@ struct Cfg {
   static constexpr int SMEM_DEN = SMEM_KS + SM_WARPS * KS_PER_WARP * 4;  // float [NQT][2][128]
   static constexpr int SMEM_PMAX = SMEM_DEN + NQT * 2 * BM * 4;     // float [NQT][2][2][128]
   static constexpr int SMEM_BAR = SMEM_PMAX + NQT * 4 * BM * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 11 * NQT;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 12 * NQT;
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
   // warps 0..: producer, one MMA issuer per query tile (then a spare warp or two),
   // then the softmax warps; any four consecutive warps cover the four TMEM lane
@@ -87,11 +91,35 @@ struct Cfg {
   static constexpr uint32_t O_COL = 0;
   static constexpr uint32_t S_COL = NQT * D;
   static constexpr uint32_t P_COL = S_COL + NQT * BN;
+  static constexpr uint32_t Q_COL = P_COL + NQT * 2 * (BN / 4);   // Q[NQT] (D/4 each)
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(P_COL + NQT * 2 * (BN / 4) <= TMEM_COLS, "tensor memory budget");
+  static_assert(Q_COL + (Q_TMEM ? NQT * (D / 4) : 0) <= TMEM_COLS, "tensor memory budget");
   static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
   static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
 };
+
+// Bytes b0 .. b0+127 of query row n (head bh) into 32 tensor-memory columns at taddr
+// (this warp's lanes), four bytes per column in order; rows past Nq are zero.
+__device__ __forceinline__ void store_q_row(const FwdParams& p, int bh, int n, int D, int b0,
+                                            uint32_t taddr) {
+  uint32_t r[32];
+  if (n < p.Nq) {
+    const uint4* src =
+        reinterpret_cast<const uint4*>(p.q8 + (static_cast<int64_t>(bh) * p.Nq + n) * D + b0);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = __ldg(src + c);
+      r[4 * c] = v.x;
+      r[4 * c + 1] = v.y;
+      r[4 * c + 2] = v.z;
+      r[4 * c + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) r[c] = 0u;
+  }
+  tmem_st32(taddr, r);
+}
 
 template <int D, int NQT, int KMODE>
 __global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
@@ -120,6 +148,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax: PV_i(t) done
   uint64_t* drain = pv_done + 2 * NQT;
   uint64_t* pair_bar = drain + NQT;          // [NQT][4] the two halves of a row quadrant: tile maximum
+  uint64_t* q_ready = pair_bar + 4 * NQT;    // [NQT] softmax -> MMA: Q_i stored in tensor memory
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -152,6 +181,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       mbar_init(s_free + i, C::ARRIVALS);             // one lane per softmax warp
       for (int q = 0; q < 4; ++q) mbar_init(pair_bar + i * 4 + q, 2);
+      mbar_init(q_ready + i, C::ARRIVALS);            // one lane per softmax warp
     }
     for (int i = 0; i < NQT; ++i) mbar_init(drain + i, 1);
     fence_barrier_init();
@@ -172,11 +202,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nvalid * C::Q_BYTES));
-      for (int i = 0; i < nvalid; ++i)
-        for (int ch = 0; ch < C::NCH; ++ch)
-          tma_load_3d(smem + C::SMEM_Q + i * C::Q_BYTES + ch * (BM * C::KCH), &tmQ, q_full,
-                      ch * C::KCH, (qt0 + i) * BM, bh);
+      if (!C::Q_TMEM) {
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nvalid * C::Q_BYTES));
+        for (int i = 0; i < nvalid; ++i)
+          for (int ch = 0; ch < C::NCH; ++ch)
+            tma_load_3d(smem + C::SMEM_Q + i * C::Q_BYTES + ch * (BM * C::KCH), &tmQ, q_full,
+                        ch * C::KCH, (qt0 + i) * BM, bh);
+      }
       int issued = 0;
       for (int t = 0; t < nK; ++t) {
         const int s = t % C::STAGES;
@@ -195,7 +227,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         issued = t + 1;
       }
       int dummy = 0;      // drain: every issued copy must land before the CTA may exit
-      mbar_wait(q_full, 0, &dummy, p.dev_err, kErrTimeoutDrain);
+      if (!C::Q_TMEM) mbar_wait(q_full, 0, &dummy, p.dev_err, kErrTimeoutDrain);
       for (int u = max(0, issued - C::STAGES); u < issued; ++u)
         if (u != p.stall_tile)
           mbar_wait(kv_full + (u % C::STAGES), (u / C::STAGES) & 1, &dummy, p.dev_err,
@@ -217,15 +249,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
-          const uint64_t ad = smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
           // split layout: the first K step overwrites S; full rows: onto the kMagic bits
-          mma_i8_ss(tS, ad, bd, C::IDESC_QK, (C::SPLIT && kk == 0) ? 0u : 1u);
+          const uint32_t acc = (C::SPLIT && kk == 0) ? 0u : 1u;
+          if constexpr (C::Q_TMEM)   // Q_i row r in lane r, 4 bytes per column, 8 columns per K step
+            mma_i8_ts(tS, tmem + C::Q_COL + i * (D / 4) + kk * 8, bd, C::IDESC_QK, acc);
+          else
+            mma_i8_ss(tS, smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK), bd,
+                      C::IDESC_QK, acc);
         }
         tc_commit(s_full + i);
       };
-      bool ok = mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ) &&
+      bool ok = (C::Q_TMEM ? mbar_wait(q_ready + i, 0, abort, p.dev_err, kErrTimeoutQ)
+                           : mbar_wait(q_full, 0, abort, p.dev_err, kErrTimeoutQ)) &&
                 mbar_wait(kv_full, 0, abort, p.dev_err, kErrTimeoutKV) &&
                 mbar_wait(s_free + i, 0, abort, p.dev_err, kErrTimeoutS);
       if (ok) {
@@ -293,6 +330,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         };
         float kone_next = 0.0f;
         if constexpr (KMODE == 1) kone_next = load_kone(0);
+        if constexpr (C::Q_TMEM) {   // this warp's rows, its half of the D bytes
+          store_q_row(p, bh, qt * BM + row, D, hf * 128, tmem + lane_off + C::Q_COL + i * (D / 4) + hf * 32);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_ready + i);
+        }
         // s_free phase t: QK_i(t) may overwrite S_i (phase 0 needs nothing read)
         if (lane == 0) mbar_arrive(s_free + i);
         for (int t = 0; ok && t < nK; ++t) {
@@ -492,6 +536,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         };
         float2 kpair_next = make_float2(0.0f, 0.0f);
         if constexpr (KMODE == 1) kpair_next = load_kpair(0);
+        if constexpr (C::Q_TMEM) {   // this warp's rows of Q_i (D = 128: 32 columns)
+          static_assert(!C::Q_TMEM || D == 128, "one 32-column store per row");
+          store_q_row(p, bh, qt * BM + row, D, 0, tmem + lane_off + C::Q_COL + wg * (D / 4));
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_ready + wg);
+        }
         // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
         // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
         // conversion is needed.
@@ -776,7 +828,7 @@ cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* 
     return cudaErrorInvalidValue;
   }
   FwdParams p{};
-  p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale; p.out = out; p.dev_err = dev_err;
+  p.q8 = q8; p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale; p.out = out; p.dev_err = dev_err;
   p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
   p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
   p.c = c;

@@ -11,8 +11,10 @@
 // Blackwell mapping (one CTA = NQT query tiles of 128 rows of one (b, h)):
 //   warp 0      TMA producer: Q tiles once, then K/V tiles into a STAGES ring
 //   warp 1+i    single-thread tcgen05.mma issuer of query tile i: QK^T as
-//               kind::i8 (M=128, N=64, K=32 steps) into TMEM S[i] as soon as the
-//               softmax warps have read S[i], then P.V as kind::f8f6f4 with P
+//               kind::i8 (M=128, N=64, K=32 steps; for D >= 128 the Q tile is
+//               operand A in TMEM, stored there once by the softmax warps) into
+//               TMEM S[i] as soon as the softmax warps have read S[i], then P.V
+//               as kind::f8f6f4 with P
 //               read from TMEM (M=128, N=D, K=32) accumulating into TMEM O[i]
 //   warps 4..   D <= 128: one 128-thread softmax warpgroup per query tile;
 //               thread r owns query row r (TMEM lane r): tcgen05.ld of its 64

@@ -9,7 +9,7 @@
 //   out = bf16(O * rcp(d) * v_scale)
 //
 // Blackwell mapping (one CTA = NQT query tiles of 128 rows of one (b, h)):
-//   warp 0      TMA producer: Q tiles once, then K/V tiles into a STAGES ring
+//   warp 0      TMA producer: (D = 64) the Q tiles once, K/V tiles into a STAGES ring
 //   warp 1+i    single-thread tcgen05.mma issuer of query tile i: QK^T as
 //               kind::i8 (M=128, N=64, K=32 steps; for D >= 128 the Q tile is
 //               operand A in TMEM, stored there once by the softmax warps) into

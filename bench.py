@@ -307,13 +307,23 @@ def run_gpu(args):
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
     value = sum_over_ranks(flops, dist, dev) / (ms_step / 1e3) / 1e12
 
-    # ---- end-to-end: pinned host QKV in, host output back, every step
+    # ---- end-to-end: pinned host QKV in, host output back, every step, through
+    # qattn_attention_host (chunks of KV heads overlap PCIe with compute)
     out_host = torch.empty(pipe.out.shape, dtype=torch.bfloat16).pin_memory()
+    if w.qkv is not None:
+        hview = host_qkv.view(w.B, w.Nq, 3, w.Hq, w.D)
+        hq, hk, hv = hview[:, :, 0], hview[:, :, 1], hview[:, :, 2]
+    else:
+        nq, nk = w.q.size, w.k.size
+        hq = host_qkv[:nq].view(w.q.shape)
+        hk = host_qkv[nq:nq + nk].view(w.k.shape)
+        hv = host_qkv[nq + nk:].view(w.v.shape)
+    runner = None if args.no_e2e else qa.HostRunner(
+        w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, hadamard=w.hadamard,
+        kv_heads_per_chunk=args.e2e_chunk, device=dev)
 
     def e2e_step():
-        qkv.copy_(host_qkv, non_blocking=True)
-        step()
-        out_host.copy_(pipe.out, non_blocking=True)
+        runner.run(hq, hk, hv, out_host, qw, kw, w.eps, w.rotary_dim, w.theta, stream=stream)
 
     e2e_ms = None
     if not args.no_e2e:
@@ -329,7 +339,7 @@ def run_gpu(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
-        pipe.check()
+        runner.check(stream)
 
     if rank == 0:
         peaks = {}
@@ -364,6 +374,7 @@ def run_gpu(args):
                          "algorithmic_work": "4*B*H*N^2*D = %.4e ops per launch" % flops},
             "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12 if e2e_ms else None,
                     "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "call": "qattn_attention_host, %d KV heads per chunk" % (runner.chunk if runner else 0),
                     "h2d_bytes_per_step": host_qkv.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2},
             "gpu_launches": (3 if w.hadamard else 5) * args.steps,
@@ -386,6 +397,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunk", type=int, default=None,
+                    help="KV heads per chunk of the end-to-end call (default Hkv // 8)")
     ap.add_argument("--config", default="canonical",
                     choices=["canonical", "small", "mid", "encoder", "gqa_chunk", "profile16k"],
                     help="workload; only 'canonical' is the benchmark line, the others are "

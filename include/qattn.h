@@ -187,6 +187,50 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
                           const int32_t* tiles, int n_tiles, int32_t* s_out,
                           int* dev_err, void* stream);
 
+/* ---------------------------------------------------------------- host to host
+ * The whole path for inputs and output in HOST memory, overlapping PCIe with
+ * compute.  The pages' problem is one call from BF16 Q/K/V to BF16 output; every
+ * (batch, KV head) in it is independent (per-head RMSNorm, K mean, scales and
+ * softmax), so this entry point cuts the KV heads into chunks of
+ * kv_heads_per_chunk (each with its Hq/Hkv query heads) and streams them through
+ * two device buffer sets in `workspace`: chunk c's Q/K/V go host -> device on
+ * h2d_stream while chunk c-1 computes on `stream` (qattn_prep -> qattn_quant ->
+ * qattn_fwd, or qattn_quant_hadamard -> qattn_fwd with k_scale_mode 1) and chunk
+ * c-2's output goes device -> host on d2h_stream.  The result is the same as
+ * those entry points give on the whole problem, bit for bit.  The pages have no
+ * counterpart for the chunking: an interface choice of this library.
+ * Arguments
+ *   q, k, v       BF16 views of HOST memory (pinned, for the copies to overlap):
+ *                 q [B,Nq,Hq,D], k and v [B,Nkv,Hkv,D], with stride[3] == 1 and
+ *                 stride[2] == D (whole heads back to back in a row; the
+ *                 interleaved QKV layout qualifies), rows 16-byte aligned
+ *   q_weight, k_weight, eps, rotary_dim, rope_theta   as qattn_prep (device weights;
+ *                 positions 0..N-1); unused when hadamard == 1
+ *   hadamard      0: prep + qattn_quant (Nq must equal Nkv); 1: qattn_quant_hadamard
+ *   sm_scale      as qattn_fwd
+ *   out           HOST BF16 [B,Nq,Hq,D], contiguous, 16-byte aligned
+ *   kv_heads_per_chunk  >= 1 (values above Hkv mean one chunk)
+ *   workspace     device, 256-byte aligned, >= qattn_host_workspace_bytes(...)
+ *   dev_err       as qattn_fwd (shared by all chunks)
+ *   stream        compute stream; when the call returns, all of its work
+ *                 (copies included) is ordered before anything queued on
+ *                 `stream` later, so qattn_check(dev_err, stream) ends it
+ *   h2d_stream, d2h_stream   copy streams (NULL: use `stream`, no overlap); they
+ *                 first wait for the work already queued on `stream`
+ * Ownership: the caller owns every buffer and the streams; the call creates and
+ * releases its own CUDA events.  Errors: NULL, SHAPE, STRIDE, UNSUPPORTED,
+ * WORKSPACE, CUDA, and those of the entry points it calls.  An error after the
+ * first chunk was queued leaves `out` undefined (earlier chunks may still land). */
+size_t qattn_host_workspace_bytes(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                                  int kv_heads_per_chunk);
+qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                                  qattn_bnhd q, qattn_bnhd k, qattn_bnhd v,
+                                  const uint16_t* q_weight, const uint16_t* k_weight, float eps,
+                                  int rotary_dim, double rope_theta, int hadamard, float sm_scale,
+                                  uint16_t* out, int kv_heads_per_chunk, void* workspace,
+                                  size_t workspace_bytes, int* dev_err, void* stream,
+                                  void* h2d_stream, void* d2h_stream);
+
 /* ---------------------------------------------------------------- status
  * Synchronize `stream`, read the device error word and map it: 0 -> QATTN_OK,
  * a timed-out wait -> QATTN_ERR_TIMEOUT; a CUDA error -> QATTN_ERR_CUDA. */

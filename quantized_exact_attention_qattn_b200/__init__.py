@@ -9,14 +9,15 @@ from __future__ import annotations
 
 import math
 
-from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_check,  # noqa: F401
-                   qattn_debug_stall_kv_tile, qattn_fwd, qattn_prep, qattn_quant,
-                   qattn_quant_hadamard, qattn_quant_noalloc, qattn_quant_workspace_bytes,
-                   qattn_scores, qattn_version)
+from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_attention_host,  # noqa: F401
+                   qattn_check, qattn_debug_stall_kv_tile, qattn_fwd, qattn_host_workspace_bytes,
+                   qattn_prep, qattn_quant, qattn_quant_hadamard, qattn_quant_noalloc,
+                   qattn_quant_workspace_bytes, qattn_scores, qattn_version)
 
-__all__ = ["Pipeline", "QAttnError", "qattn_prep", "qattn_quant", "qattn_quant_noalloc",
-           "qattn_quant_hadamard",
+__all__ = ["Pipeline", "HostRunner", "QAttnError", "qattn_prep", "qattn_quant",
+           "qattn_quant_noalloc", "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
+           "qattn_host_workspace_bytes", "qattn_attention_host",
            "qattn_debug_stall_kv_tile", "qattn_version", "load"]
 
 
@@ -96,6 +97,47 @@ class Pipeline:
     @property
     def attn_ops(self) -> float:
         return 4.0 * self.B * self.Hq * self.Nq * self.Nkv * self.D
+
+
+class HostRunner:
+    """``qattn_attention_host`` with its device workspace, error word and two
+    copy streams: host Q/K/V in, host output back, chunks of KV heads overlapping
+    PCIe with compute.  Default chunk (measured on one B200): inputs of 512 MB or
+    more in about fourteen chunks (4 KV heads at N37810 H56 D128: 40.9 ms against
+    41.9 with 7 and 46.0 with 14), smaller ones in about four of at least two KV
+    heads (encoder B32 N729 H16 D64: 3.21 ms against 3.76 in one chunk; GQA
+    Nq1024 Nkv32768 Hkv4 D256: 3.53 ms with two heads, 3.68 with one chunk, 3.88
+    with one head per chunk)."""
+
+    def __init__(self, B, Nq, Nkv, Hq, Hkv, D, *, hadamard=False, kv_heads_per_chunk=None,
+                 device="cuda"):
+        import torch
+        self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D = B, Nq, Nkv, Hq, Hkv, D
+        self.hadamard = hadamard
+        in_bytes = 2 * B * D * (Nq * Hq + 2 * Nkv * Hkv)
+        if in_bytes >= (512 << 20):
+            default = -(-Hkv // 14)
+        else:
+            default = max(-(-Hkv // 4), 2 if Hkv >= 4 else 1)
+        self.chunk = kv_heads_per_chunk or default
+        nbytes = qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, self.chunk)
+        if nbytes == 0:
+            raise ValueError("invalid sizes for qattn_host_workspace_bytes")
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.h2d = torch.cuda.Stream(device=device)
+        self.d2h = torch.cuda.Stream(device=device)
+
+    def run(self, q, k, v, out, q_weight=None, k_weight=None, eps=1e-5, rotary_dim=0,
+            theta=10000.0, sm_scale=0.0, stream=None):
+        """q, k, v: host BF16 [B, N, H, D] views (pinned); out: host BF16 [B, Nq, Hq, D]."""
+        qattn_attention_host(self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D, q, k, v,
+                             q_weight, k_weight, eps, rotary_dim, theta, self.hadamard, sm_scale,
+                             out, self.chunk, self.ws, self.dev_err, stream, self.h2d, self.d2h)
+        return out
+
+    def check(self, stream=None):
+        qattn_check(self.dev_err, stream)
 
 
 def default_sm_scale(D: int) -> float:

@@ -21,8 +21,8 @@ QATTN_STATUS = {0: "QATTN_OK", 1: "QATTN_ERR_NULL", 2: "QATTN_ERR_SHAPE", 3: "QA
 
 EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_noalloc",
             "qattn_quant_hadamard",
-            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_debug_stall_kv_tile",
-            "qattn_last_error", "qattn_version")
+            "qattn_fwd", "qattn_scores", "qattn_host_workspace_bytes", "qattn_attention_host",
+            "qattn_check", "qattn_debug_stall_kv_tile", "qattn_last_error", "qattn_version")
 
 
 class QAttnError(RuntimeError):
@@ -62,12 +62,16 @@ def load(path: str | None = None) -> ctypes.CDLL:
                                          vp, vp, sz, vp]
     lib.qattn_fwd.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, vp, vp]
     lib.qattn_scores.argtypes = [i, i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
+    lib.qattn_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    lib.qattn_host_workspace_bytes.restype = sz
+    lib.qattn_attention_host.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, f32, i, f64,
+                                         i, f32, vp, i, vp, sz, vp, vp, vp, vp]
     lib.qattn_check.argtypes = [vp, vp]
     lib.qattn_debug_stall_kv_tile.argtypes = [i]
     lib.qattn_last_error.restype = ctypes.c_char_p
     lib.qattn_version.restype = ctypes.c_char_p
     for name in ("qattn_prep", "qattn_quant", "qattn_quant_noalloc", "qattn_quant_hadamard", "qattn_fwd",
-                 "qattn_scores", "qattn_check", "qattn_debug_stall_kv_tile"):
+                 "qattn_scores", "qattn_attention_host", "qattn_check", "qattn_debug_stall_kv_tile"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -145,6 +149,25 @@ def qattn_fwd(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v8
 def qattn_scores(B, Nq, Nkv, Hq, Hkv, D, q8, k8, tiles, n_tiles, s_out, dev_err, stream=None):
     _check(load().qattn_scores(B, Nq, Nkv, Hq, Hkv, D, _ptr(q8), _ptr(k8), _ptr(tiles), n_tiles,
                                _ptr(s_out), _ptr(dev_err), _stream(stream)))
+
+
+def qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, kv_heads_per_chunk) -> int:
+    return int(load().qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, kv_heads_per_chunk))
+
+
+def qattn_attention_host(B, Nq, Nkv, Hq, Hkv, D, q, k, v, q_weight, k_weight, eps, rotary_dim,
+                         rope_theta, hadamard, sm_scale, out, kv_heads_per_chunk, workspace,
+                         dev_err, stream=None, h2d_stream=None, d2h_stream=None,
+                         workspace_bytes=None):
+    """q, k, v, out: HOST tensors (pinned); workspace, dev_err, weights: device.
+    h2d_stream / d2h_stream None: the copies run on `stream` (no overlap)."""
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    copy = lambda st: None if st is None else _stream(st)
+    _check(load().qattn_attention_host(B, Nq, Nkv, Hq, Hkv, D, bnhd(q), bnhd(k), bnhd(v),
+                                       _ptr(q_weight), _ptr(k_weight), eps, rotary_dim, rope_theta,
+                                       int(hadamard), sm_scale, _ptr(out), kv_heads_per_chunk,
+                                       _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream),
+                                       copy(h2d_stream), copy(d2h_stream)))
 
 
 def qattn_check(dev_err, stream=None):

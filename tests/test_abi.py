@@ -123,3 +123,34 @@ def test_stall_hook_refuses_negative_tiles_and_resets(lib):
     assert lib.qattn_debug_stall_kv_tile(-2) == 2          # QATTN_ERR_SHAPE
     assert "kv_tile" in lib.qattn_last_error().decode() or "tile" in lib.qattn_last_error().decode()
     assert lib.qattn_debug_stall_kv_tile(-1) == 0          # off (the initial state)
+
+
+def test_host_pipeline_workspace_query_and_refusals(lib):
+    ws = lib.qattn_host_workspace_bytes
+    one = ws(1, 37810, 37810, 56, 56, 128, 7)
+    # two buffer sets, each at least the chunk's BF16 Q/K/V, prepared Q/K and output
+    assert one >= 2 * 6 * 37810 * 7 * 128 * 2
+    assert ws(1, 37810, 37810, 56, 56, 128, 56) == ws(1, 37810, 37810, 56, 56, 128, 500)
+    assert ws(1, 37810, 37810, 56, 56, 128, 8) > one
+    assert ws(1, 100, 100, 4, 3, 128, 1) == 0        # Hq % Hkv
+    assert ws(1, 100, 100, 4, 4, 96, 1) == 0         # head dim
+    assert ws(1, 100, 100, 4, 4, 128, 0) == 0        # chunk
+    need = ws(1, 256, 256, 2, 2, 128, 1)
+    ALIGNED = 0x7f0000010000
+
+    def call(q=None, k=None, v=None, Nq=256, hadamard=0, chunk=1, out=FAKE, ws_ptr=ALIGNED,
+             nbytes=need, err=FAKE):
+        view = _view(strides=(256 * 2 * 128, 2 * 128, 128, 1))
+        return lib.qattn_attention_host(1, Nq, 256, 2, 2, 128, q or view, k or view, v or view,
+                                        None, None, 1e-5, 0, 10000.0, hadamard, 0.0, out, chunk,
+                                        ws_ptr, nbytes, err, None, None, None)
+    assert call(chunk=0) == 2
+    assert call(hadamard=2) == 4
+    assert call(Nq=128) == 4 and "Nq == Nkv" in lib.qattn_last_error().decode()
+    assert call(q=_view(ptr=0)) == 1
+    assert call(k=_view(strides=(256 * 4 * 128, 4 * 128, 256, 1))) == 3   # heads not back to back
+    assert call(out=None) == 1
+    assert call(err=None) == 1
+    assert call(out=FAKE + 8) == 3
+    assert call(nbytes=need - 1) == 5
+    assert call(ws_ptr=ALIGNED + 16) == 5

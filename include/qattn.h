@@ -194,7 +194,7 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  * softmax), so this entry point cuts the KV heads into chunks of
  * kv_heads_per_chunk (each with its Hq/Hkv query heads) and streams them through
  * two device buffer sets in `workspace`: chunk c's Q/K/V go host -> device on
- * h2d_stream while chunk c-1 computes on `stream` (qattn_prep -> qattn_quant ->
+ * h2d_stream while chunk c-1 computes on its set's stream (qattn_prep -> qattn_quant ->
  * qattn_fwd, or qattn_quant_hadamard -> qattn_fwd with k_scale_mode 1) and chunk
  * c-2's output goes device -> host on d2h_stream.  The result is the same as
  * those entry points give on the whole problem, bit for bit.  The pages have no
@@ -209,14 +209,21 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  *   hadamard      0: prep + qattn_quant (Nq must equal Nkv); 1: qattn_quant_hadamard
  *   sm_scale      as qattn_fwd
  *   out           HOST BF16 [B,Nq,Hq,D], contiguous, 16-byte aligned
- *   kv_heads_per_chunk  >= 1 (values above Hkv mean one chunk)
+ *   kv_heads_per_chunk  >= 1: the chunk size (values above Hkv mean one chunk);
+ *                 with Hkv >= 8 * kv_heads_per_chunk the first two chunks are a
+ *                 quarter and a half of it (the first copy is then short)
  *   workspace     device, 256-byte aligned, >= qattn_host_workspace_bytes(...)
  *   dev_err       as qattn_fwd (shared by all chunks)
- *   stream        compute stream; when the call returns, all of its work
- *                 (copies included) is ordered before anything queued on
- *                 `stream` later, so qattn_check(dev_err, stream) ends it
- *   h2d_stream, d2h_stream   copy streams (NULL: use `stream`, no overlap); they
- *                 first wait for the work already queued on `stream`
+ *   stream        compute stream of buffer set 0; when the call returns, all of
+ *                 its work (copies and stream2 included) is ordered before
+ *                 anything queued on `stream` later, so qattn_check(dev_err,
+ *                 stream) ends it
+ *   stream2       compute stream of buffer set 1 (NULL: `stream`): consecutive
+ *                 chunks then overlap, the next one's kernels filling the SMs
+ *                 the previous one's last wave leaves idle
+ *   h2d_stream, d2h_stream   copy streams (NULL: use `stream`, no overlap)
+ *                 stream2, h2d_stream and d2h_stream first wait for the work
+ *                 already queued on `stream`
  * Ownership: the caller owns every buffer and the streams; the call creates and
  * releases its own CUDA events.  Errors: NULL, SHAPE, STRIDE, UNSUPPORTED,
  * WORKSPACE, CUDA, and those of the entry points it calls.  An error after the
@@ -229,7 +236,7 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                   int rotary_dim, double rope_theta, int hadamard, float sm_scale,
                                   uint16_t* out, int kv_heads_per_chunk, void* workspace,
                                   size_t workspace_bytes, int* dev_err, void* stream,
-                                  void* h2d_stream, void* d2h_stream);
+                                  void* stream2, void* h2d_stream, void* d2h_stream);
 
 /* ---------------------------------------------------------------- status
  * Synchronize `stream`, read the device error word and map it: 0 -> QATTN_OK,

@@ -125,6 +125,7 @@ class HostRunner:
             raise ValueError("invalid sizes for qattn_host_workspace_bytes")
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.compute2 = torch.cuda.Stream(device=device)
         self.h2d = torch.cuda.Stream(device=device)
         self.d2h = torch.cuda.Stream(device=device)
 
@@ -133,7 +134,8 @@ class HostRunner:
         """q, k, v: host BF16 [B, N, H, D] views (pinned); out: host BF16 [B, Nq, Hq, D]."""
         qattn_attention_host(self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D, q, k, v,
                              q_weight, k_weight, eps, rotary_dim, theta, self.hadamard, sm_scale,
-                             out, self.chunk, self.ws, self.dev_err, stream, self.h2d, self.d2h)
+                             out, self.chunk, self.ws, self.dev_err, stream, self.compute2,
+                             self.h2d, self.d2h)
         return out
 
     def check(self, stream=None):

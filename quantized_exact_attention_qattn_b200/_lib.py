@@ -65,7 +65,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
     lib.qattn_host_workspace_bytes.restype = sz
     lib.qattn_attention_host.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, f32, i, f64,
-                                         i, f32, vp, i, vp, sz, vp, vp, vp, vp]
+                                         i, f32, vp, i, vp, sz, vp, vp, vp, vp, vp]
     lib.qattn_check.argtypes = [vp, vp]
     lib.qattn_debug_stall_kv_tile.argtypes = [i]
     lib.qattn_last_error.restype = ctypes.c_char_p
@@ -157,17 +157,17 @@ def qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, kv_heads_per_chunk) -> in
 
 def qattn_attention_host(B, Nq, Nkv, Hq, Hkv, D, q, k, v, q_weight, k_weight, eps, rotary_dim,
                          rope_theta, hadamard, sm_scale, out, kv_heads_per_chunk, workspace,
-                         dev_err, stream=None, h2d_stream=None, d2h_stream=None,
+                         dev_err, stream=None, stream2=None, h2d_stream=None, d2h_stream=None,
                          workspace_bytes=None):
     """q, k, v, out: HOST tensors (pinned); workspace, dev_err, weights: device.
-    h2d_stream / d2h_stream None: the copies run on `stream` (no overlap)."""
+    stream2 / h2d_stream / d2h_stream None: that work runs on `stream`."""
     nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
     copy = lambda st: None if st is None else _stream(st)
     _check(load().qattn_attention_host(B, Nq, Nkv, Hq, Hkv, D, bnhd(q), bnhd(k), bnhd(v),
                                        _ptr(q_weight), _ptr(k_weight), eps, rotary_dim, rope_theta,
                                        int(hadamard), sm_scale, _ptr(out), kv_heads_per_chunk,
                                        _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream),
-                                       copy(h2d_stream), copy(d2h_stream)))
+                                       copy(stream2), copy(h2d_stream), copy(d2h_stream)))
 
 
 def qattn_check(dev_err, stream=None):

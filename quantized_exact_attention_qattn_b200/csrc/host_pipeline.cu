@@ -122,7 +122,7 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                   int rotary_dim, double rope_theta, int hadamard, float sm_scale,
                                   uint16_t* out, int kv_heads_per_chunk, void* workspace,
                                   size_t workspace_bytes, int* dev_err, void* stream,
-                                  void* h2d_stream, void* d2h_stream) {
+                                  void* stream2, void* h2d_stream, void* d2h_stream) {
   if (!sizes_ok(B, Nq, Nkv, Hq, Hkv, D, kv_heads_per_chunk))
     return hfail(QATTN_ERR_SHAPE,
                  "attention_host: sizes must be positive, Hq %% Hkv == 0, D in {64,128,256} and "
@@ -148,6 +148,9 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                  2 * L.bytes);
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // buffer set s computes on compute[s]: chunks of one set stay in order, and the
+  // next chunk's kernels fill the SMs that the previous chunk's last wave leaves
+  cudaStream_t compute[2] = {cs, stream2 ? static_cast<cudaStream_t>(stream2) : cs};
   cudaStream_t hs = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : cs;
   cudaStream_t ds = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : cs;
   cudaEvent_t ev[7];   // start, h2d[2], comp[2], d2h[2]
@@ -168,13 +171,26 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
   // previous call's use of the workspace included)
   cu(cudaEventRecord(e_start, cs), "cudaEventRecord") &&
       cu(cudaStreamWaitEvent(hs, e_start, 0), "cudaStreamWaitEvent") &&
-      cu(cudaStreamWaitEvent(ds, e_start, 0), "cudaStreamWaitEvent");
+      cu(cudaStreamWaitEvent(ds, e_start, 0), "cudaStreamWaitEvent") &&
+      cu(cudaStreamWaitEvent(compute[1], e_start, 0), "cudaStreamWaitEvent");
 
-  const int n_chunks = (Hkv + ck - 1) / ck;
+  // With eight or more chunks the sizes ramp up (a quarter, a half, then the full
+  // chunk): nothing computes before the first chunk has crossed PCIe, so it is
+  // made short.  Fewer, smaller problems keep equal chunks (narrow copy rows move
+  // slowly).
+  const bool ramp = Hkv >= 8 * ck;
+  auto chunk_heads = [&](int c) {
+    if (!ramp) return ck;
+    return c == 0 ? std::max(1, ck / 4) : (c == 1 ? std::max(1, ck / 2) : ck);
+  };
+  int n_chunks = 0;
+  for (int h = 0; h < Hkv; h += chunk_heads(n_chunks++)) {
+  }
   uint8_t* const ws = static_cast<uint8_t*>(workspace);
-  for (int c = 0; st == QATTN_OK && c < n_chunks; ++c) {
+  int k0 = 0;
+  for (int c = 0; st == QATTN_OK && c < n_chunks; k0 += chunk_heads(c), ++c) {
     const int s = c & 1;
-    const int k0 = c * ck, kc = std::min(ck, Hkv - k0), q0 = k0 * G, qc = kc * G;
+    const int kc = std::min(chunk_heads(c), Hkv - k0), q0 = k0 * G, qc = kc * G;
     uint8_t* const base = ws + s * L.bytes;
     // ---- host -> device: this set's inputs were last read by chunk c-2
     if (c >= 2 && !cu(cudaStreamWaitEvent(hs, e_comp[s], 0), "cudaStreamWaitEvent")) break;
@@ -183,8 +199,9 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
         cu(copy_in(base + L.v_in, v, B, Nkv, k0, kc, D, hs), "cudaMemcpy2DAsync (v)");
     if (!cu(cudaEventRecord(e_h2d[s], hs), "cudaEventRecord")) break;
     // ---- compute: inputs landed, and this set's output was copied out (chunk c-2)
-    if (!cu(cudaStreamWaitEvent(cs, e_h2d[s], 0), "cudaStreamWaitEvent")) break;
-    if (c >= 2 && !cu(cudaStreamWaitEvent(cs, e_d2h[s], 0), "cudaStreamWaitEvent")) break;
+    cudaStream_t xs = compute[s];
+    if (!cu(cudaStreamWaitEvent(xs, e_h2d[s], 0), "cudaStreamWaitEvent")) break;
+    if (c >= 2 && !cu(cudaStreamWaitEvent(xs, e_d2h[s], 0), "cudaStreamWaitEvent")) break;
     const int64_t sq[4] = {static_cast<int64_t>(Nq) * qc * D, static_cast<int64_t>(qc) * D, D, 1};
     const int64_t sk[4] = {static_cast<int64_t>(Nkv) * kc * D, static_cast<int64_t>(kc) * D, D, 1};
     const qattn_bnhd qv{base + L.q_in, {sq[0], sq[1], sq[2], sq[3]}};
@@ -199,22 +216,22 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
     if (hadamard) {
       st = qattn_quant_hadamard(B, Nq, Nkv, qc, kc, D, qv, kv, vv, q8, q_scale, k8,
                                 reinterpret_cast<uint16_t*>(base + L.k_scale), v8t, v_scale,
-                                base + L.qws, L.qws_bytes, cs);
+                                base + L.qws, L.qws_bytes, xs);
     } else {
       const qattn_bnhd qpv{base + L.qp, {sq[0], sq[1], sq[2], sq[3]}};
       const qattn_bnhd kpv{base + L.kp, {sk[0], sk[1], sk[2], sk[3]}};
       st = qattn_prep(B, Nq, qc, kc, D, qv, kv, q_weight, k_weight, eps, rotary_dim, rope_theta, 0,
-                      reinterpret_cast<uint16_t*>(base + L.qp), reinterpret_cast<uint16_t*>(base + L.kp), cs);
+                      reinterpret_cast<uint16_t*>(base + L.qp), reinterpret_cast<uint16_t*>(base + L.kp), xs);
       if (st == QATTN_OK)
         st = qattn_quant(B, Nq, Nkv, qc, kc, D, qpv, kpv, vv, q8, q_scale, k8,
                          reinterpret_cast<float*>(base + L.k_scale),
                          reinterpret_cast<float*>(base + L.k_mean), v8t, v_scale, base + L.qws,
-                         L.qws_bytes, cs);
+                         L.qws_bytes, xs);
     }
     if (st == QATTN_OK)
       st = qattn_fwd(B, Nq, Nkv, qc, kc, D, q8, q_scale, k8, base + L.k_scale, hadamard ? 1 : 0,
-                     v8t, v_scale, sm_scale, out_c, dev_err, cs);
-    if (st != QATTN_OK || !cu(cudaEventRecord(e_comp[s], cs), "cudaEventRecord")) break;
+                     v8t, v_scale, sm_scale, out_c, dev_err, xs);
+    if (st != QATTN_OK || !cu(cudaEventRecord(e_comp[s], xs), "cudaEventRecord")) break;
     // ---- device -> host: heads [q0, q0+qc) of every output row (b, n), one 2D copy
     if (!cu(cudaStreamWaitEvent(ds, e_comp[s], 0), "cudaStreamWaitEvent")) break;
     {

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   constexpr int HPW = 32 / L;  // head rows per warp
   __shared__ __align__(16) float s_cos[QATTN_PREP_TOKENS][D / 2];
   __shared__ __align__(16) float s_sin[QATTN_PREP_TOKENS][D / 2];
+  __shared__ double s_freq[D / 2];   // theta^(-2i/R), the same for every token
 
   const int tiles = (a.N + QATTN_PREP_TOKENS - 1) / QATTN_PREP_TOKENS;
   const int b = blockIdx.x / tiles;
@@ -102,10 +103,12 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   // The first loads go out before the FP64 RoPE tables of all the CTA's tokens
   // are computed (by all threads at once), so the table latency overlaps them.
   load_passes(n0, 0);
+  for (int i = threadIdx.x; i < half; i += blockDim.x)
+    s_freq[i] = pow(a.theta, -(2.0 * i) / static_cast<double>(a.rotary_dim));
+  __syncthreads();
   for (int idx = threadIdx.x; idx < nt * half; idx += blockDim.x) {
     const int k = idx / half, i = idx - k * half;
-    const double inv_freq = pow(a.theta, -(2.0 * i) / static_cast<double>(a.rotary_dim));
-    const double ang = static_cast<double>(a.pos_offset + n0 + k) * inv_freq;
+    const double ang = static_cast<double>(a.pos_offset + n0 + k) * s_freq[i];
     double sv, cv;
     sincos(ang, &sv, &cv);
     s_cos[k][i] = bf16_round_f64(cv);

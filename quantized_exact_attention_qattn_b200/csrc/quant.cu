@@ -127,32 +127,30 @@ __global__ void kv_finalize_kernel(int B, int Nkv, int nK, int C, bool has_k,
   if (idx >= static_cast<int64_t>(B) * C) return;
   const int b = static_cast<int>(idx / C), c = static_cast<int>(idx - static_cast<int64_t>(b) * C);
   const size_t base = static_cast<size_t>(b) * nK * C + c;
-  // loads are issued 16 blocks ahead of the (strictly ascending) additions
-  if (has_k) {
-    double s = 0.0;
-    int j = 0;
-    for (; j + 16 <= nK; j += 16) {
-      double v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = ksum[base + static_cast<size_t>(j + u) * C];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) s = __dadd_rn(s, v[u]);
-    }
-    for (; j < nK; ++j) s = __dadd_rn(s, ksum[base + static_cast<size_t>(j) * C]);
-    k_mean[idx] = __double2float_rn(__ddiv_rn(s, static_cast<double>(Nkv)));
-  }
+  // loads of K sums and V maxima are issued together, 16 blocks ahead of the
+  // (strictly ascending) additions
+  double s = 0.0;
   float a = 0.0f;
-  {
-    int j = 0;
-    for (; j + 16 <= nK; j += 16) {
-      float v[16];
+  int j = 0;
+  for (; j + 16 <= nK; j += 16) {
+    double ks[16];
+    float vm[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = vmax[base + static_cast<size_t>(j + u) * C];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) a = fmaxf(a, v[u]);
+    for (int u = 0; u < 16; ++u) {
+      if (has_k) ks[u] = ksum[base + static_cast<size_t>(j + u) * C];
+      vm[u] = vmax[base + static_cast<size_t>(j + u) * C];
     }
-    for (; j < nK; ++j) a = fmaxf(a, vmax[base + static_cast<size_t>(j) * C]);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (has_k) s = __dadd_rn(s, ks[u]);
+      a = fmaxf(a, vm[u]);
+    }
   }
+  for (; j < nK; ++j) {
+    if (has_k) s = __dadd_rn(s, ksum[base + static_cast<size_t>(j) * C]);
+    a = fmaxf(a, vmax[base + static_cast<size_t>(j) * C]);
+  }
+  if (has_k) k_mean[idx] = __double2float_rn(__ddiv_rn(s, static_cast<double>(Nkv)));
   a = fmaxf(1e-7f, a);
   v_scale[idx] = __fdiv_rn(a, 2.25f);
   vfac[idx] = __fdiv_rn(2.25f, a);

@@ -143,7 +143,7 @@ def test_host_pipeline_workspace_query_and_refusals(lib):
         view = _view(strides=(256 * 2 * 128, 2 * 128, 128, 1))
         return lib.qattn_attention_host(1, Nq, 256, 2, 2, 128, q or view, k or view, v or view,
                                         None, None, 1e-5, 0, 10000.0, hadamard, 0.0, out, chunk,
-                                        ws_ptr, nbytes, err, None, None, None)
+                                        ws_ptr, nbytes, err, None, None, None, None)
     assert call(chunk=0) == 2
     assert call(hadamard=2) == 4
     assert call(Nq=128) == 4 and "Nq == Nkv" in lib.qattn_last_error().decode()

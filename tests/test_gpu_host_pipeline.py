@@ -33,7 +33,7 @@ def run_host(w, chunk, copy_streams=True):
     runner = qa.HostRunner(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, hadamard=w.hadamard,
                            kv_heads_per_chunk=chunk, device=DEV)
     if not copy_streams:
-        runner.h2d = runner.d2h = None
+        runner.compute2 = runner.h2d = runner.d2h = None
     out = torch.empty((w.B, w.Nq, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
     out.view(torch.int16).fill_(0x7fc0)                      # NaN sentinel: every element is written
     qw = dev_bf16(w.q_weight) if w.q_weight is not None else None
@@ -50,6 +50,15 @@ def test_host_pipeline_equals_device_pipeline(chunk):
     got = run_host(w, chunk)
     ref = run_pipeline(w).out.cpu()
     assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), chunk
+
+
+def test_host_pipeline_ramped_chunks():
+    # 16 KV heads in chunks of 2: eight or more chunks, so the first two are
+    # shortened (1 and 1 heads) and the rest follow at 2
+    w = synth.custom(31, 1, 700, 16, 128)
+    got = run_host(w, 2)
+    ref = run_pipeline(w).out.cpu()
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
 
 
 def test_host_pipeline_interleaved_inputs_and_serial_copies():

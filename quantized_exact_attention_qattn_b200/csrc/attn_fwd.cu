@@ -573,6 +573,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
           tmem_wait_ld();
           reset_s(tS, magic);                             // reset S for QK_i(t+1)
+          // release S right away: the next QK is on this warp's critical path, the
+          // store latency is short next to the max tree it would otherwise follow
+          tmem_wait_st();                                 // the reset of S has landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + wg);
           const bool last = (t == nK - 1);
           float mn;
           float2 a2, nb2;
@@ -631,10 +637,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
             nb2 = make_float2(-mn, -mn);
           }
-          tmem_wait_st();                                 // the reset of S has landed
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_free + wg);
           const float old = ex2_approx(__fsub_rn(m, mn));
           if constexpr (KMODE == 0) {
             exp_block<0, 64>(x, a2, nb2);

@@ -36,11 +36,11 @@ WORKLOAD = {"workload": "canonical interleaved-QKV quantized attention prefill",
             "l2": "inputs larger than L2 (1.63 GB QKV, 126 MB L2); no flush needed"}
 NOMINAL_FP8_OVER_BF16 = 2.0          # 4.5 / 2.25 PFLOP/s dense (nominal ratio)
 # DRAM bytes per canonical attention launch: ncu dram__bytes_read + write on the
-# B1 N16384 H32 D128 case (202.6 MB + 102.0 MB = 304.6 MB) scaled by the units
+# B1 N16384 H32 D128 case (201.5 MB + 102.5 MB = 304.1 MB) scaled by the units
 # processed (N*H: 2117360 / 524288 = 4.0386).  Valid only for the attention kernel
 # the capture was taken on (this file's kernel as of the capture); set to None when
 # the kernel changes and re-take the capture.
-ATTN_TRAFFIC_BYTES = int((202612992 + 102009088) * 2117360 / 524288)
+ATTN_TRAFFIC_BYTES = int((201517312 + 102539520) * 2117360 / 524288)
 SPEC_FP8_TFLOPS = 4500.0
 
 

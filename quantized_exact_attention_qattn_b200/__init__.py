@@ -14,7 +14,7 @@ from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_attention_host,  # no
                    qattn_prep, qattn_quant, qattn_quant_hadamard, qattn_quant_noalloc,
                    qattn_quant_workspace_bytes, qattn_scores, qattn_version)
 
-__all__ = ["Pipeline", "HostRunner", "QAttnError", "qattn_prep", "qattn_quant",
+__all__ = ["Pipeline", "HostRunner", "default_kv_heads_per_chunk", "QAttnError", "qattn_prep", "qattn_quant",
            "qattn_quant_noalloc", "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
            "qattn_host_workspace_bytes", "qattn_attention_host",
@@ -99,27 +99,30 @@ class Pipeline:
         return 4.0 * self.B * self.Hq * self.Nq * self.Nkv * self.D
 
 
+def default_kv_heads_per_chunk(B, Nq, Nkv, Hq, Hkv, D) -> int:
+    """KV heads per chunk for ``qattn_attention_host`` (measured on one B200):
+    inputs of 512 MB or more in about fourteen chunks (4 KV heads at N37810 H56
+    D128: 40.9 ms end to end against 41.9 with 7 and 46.0 with 14), smaller ones
+    in about four chunks of at least two KV heads (encoder B32 N729 H16 D64: 3.21
+    ms against 3.76 in one chunk; GQA Nq1024 Nkv32768 Hkv4 D256: 3.53 ms with two
+    heads, 3.68 in one chunk, 3.88 with one head per chunk)."""
+    in_bytes = 2 * B * D * (Nq * Hq + 2 * Nkv * Hkv)
+    if in_bytes >= (512 << 20):
+        return -(-Hkv // 14)
+    return min(Hkv, max(-(-Hkv // 4), 2 if Hkv >= 4 else 1))
+
+
 class HostRunner:
     """``qattn_attention_host`` with its device workspace, error word and two
     copy streams: host Q/K/V in, host output back, chunks of KV heads overlapping
-    PCIe with compute.  Default chunk (measured on one B200): inputs of 512 MB or
-    more in about fourteen chunks (4 KV heads at N37810 H56 D128: 40.9 ms against
-    41.9 with 7 and 46.0 with 14), smaller ones in about four of at least two KV
-    heads (encoder B32 N729 H16 D64: 3.21 ms against 3.76 in one chunk; GQA
-    Nq1024 Nkv32768 Hkv4 D256: 3.53 ms with two heads, 3.68 with one chunk, 3.88
-    with one head per chunk)."""
+    PCIe with compute; the default chunk is ``default_kv_heads_per_chunk``."""
 
     def __init__(self, B, Nq, Nkv, Hq, Hkv, D, *, hadamard=False, kv_heads_per_chunk=None,
                  device="cuda"):
         import torch
         self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D = B, Nq, Nkv, Hq, Hkv, D
         self.hadamard = hadamard
-        in_bytes = 2 * B * D * (Nq * Hq + 2 * Nkv * Hkv)
-        if in_bytes >= (512 << 20):
-            default = -(-Hkv // 14)
-        else:
-            default = max(-(-Hkv // 4), 2 if Hkv >= 4 else 1)
-        self.chunk = kv_heads_per_chunk or default
+        self.chunk = kv_heads_per_chunk or default_kv_heads_per_chunk(B, Nq, Nkv, Hq, Hkv, D)
         nbytes = qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, self.chunk)
         if nbytes == 0:
             raise ValueError("invalid sizes for qattn_host_workspace_bytes")

@@ -154,3 +154,15 @@ def test_host_pipeline_workspace_query_and_refusals(lib):
     assert call(out=FAKE + 8) == 3
     assert call(nbytes=need - 1) == 5
     assert call(ws_ptr=ALIGNED + 16) == 5
+
+
+def test_default_host_chunk_rule():
+    f = qa.default_kv_heads_per_chunk
+    assert f(1, 37810, 37810, 56, 56, 128) == 4        # 1.63 GB of input: ~14 chunks
+    assert f(1, 1024, 32768, 16, 4, 256) == 2          # 143 MB, GQA: two heads per chunk
+    assert f(32, 729, 729, 16, 16, 64) == 4            # 143 MB: four chunks
+    assert f(1, 256, 256, 2, 2, 128) == 1              # two KV heads: one per chunk
+    assert f(1, 256, 256, 1, 1, 128) == 1
+    for args in [(1, 37810, 37810, 56, 56, 128), (2, 5000, 5000, 8, 2, 128), (1, 9000, 9000, 3, 3, 64)]:
+        c = f(*args)
+        assert 1 <= c <= args[4]

@@ -403,6 +403,34 @@ def test_gqa_maps_query_head_to_kv_head_by_division():
     assert np.array_equal(out, out2)
 
 
+def test_per_token_scales_equal_to_the_block_scale_reproduce_block_mode():
+    # "Q And K Quantization" scales K per 64-row block; the rotated variant scales it
+    # per token.  With every token's FP16 scale equal to its block's scale (values
+    # exact in FP16), A = (q_scale * k_scale) * c is the same number per key, so the
+    # per-token path must give the per-block output bit for bit (ragged last tile).
+    rng = np.random.default_rng(16)
+    d, nq, nkv = 64, 70, 150
+    nk = -(-nkv // 64)
+    q8 = rng.integers(-127, 128, (1, 2, nq, d)).astype(np.int8)
+    qs = (0.01 + 0.01 * rng.random((1, 2, 4))).astype(np.float32)
+    k8 = rng.integers(-127, 128, (1, 1, nkv, d)).astype(np.int8)
+    ks = (2.0 ** -7 * (1 + rng.integers(0, 8, (1, 1, nk)) / 8.0)).astype(np.float32)
+    ks_tok = np.repeat(ks, 64, axis=2)[:, :, :nkv]
+    ks16 = ks_tok.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ks16.view(np.float16).astype(np.float32), ks_tok)   # exact in FP16
+    v8t = rng.integers(0, 0x7E, (1, 1, d, 64 * nk)).astype(np.uint8)
+    vs = (0.1 + rng.random((1, 1, d))).astype(np.float32)
+    block, mb, db = O.attention(q8, qs, k8, ks, v8t, vs, nkv, k_scale_mode=0)
+    token, mt, dt = O.attention(q8, qs, k8, ks16, v8t, vs, nkv, k_scale_mode=1)
+    assert np.array_equal(block, token)
+    assert np.array_equal(mb, mt) and np.array_equal(db, dt)
+    # and a per-token scale that differs inside a block changes the output
+    ks16b = ks16.copy()
+    ks16b[0, 0, 3] = np.float16(ks_tok[0, 0, 3] * 2).view(np.uint16)
+    other, _, _ = O.attention(q8, qs, k8, ks16b, v8t, vs, nkv, k_scale_mode=1)
+    assert not np.array_equal(block, other)
+
+
 def test_row_sample_is_exact():
     w = synth.custom(22, 1, 300, 2, 64, rope=False)
     q8, qs = O.quant_q(w.q)

@@ -431,6 +431,25 @@ def test_per_token_scales_equal_to_the_block_scale_reproduce_block_mode():
     assert not np.array_equal(block, other)
 
 
+def test_v_scale_is_applied_per_output_channel():
+    # "Finalization And Tails": out[d] = bf16((O[d] / l) * v_scale[d]).  A power of two
+    # 2^e_d on v_scale[d] commutes with every rounding, so output channel d (and only
+    # it) moves by exactly 2^e_d: the scale is applied on the right axis.
+    rng = np.random.default_rng(17)
+    d, n = 64, 100
+    q8 = rng.integers(-127, 128, (1, 1, n, d)).astype(np.int8)
+    qs = (0.01 + 0.01 * rng.random((1, 1, 4))).astype(np.float32)
+    k8 = rng.integers(-127, 128, (1, 1, n, d)).astype(np.int8)
+    ks = (0.01 + 0.01 * rng.random((1, 1, 2))).astype(np.float32)
+    v8t = rng.integers(0, 0x7E, (1, 1, d, 128)).astype(np.uint8)
+    vs = (0.1 + rng.random((1, 1, d))).astype(np.float32)
+    e = rng.integers(-3, 4, d)
+    base, _, _ = O.attention(q8, qs, k8, ks, v8t, vs, n)
+    moved, _, _ = O.attention(q8, qs, k8, ks, v8t, (vs * 2.0 ** e).astype(np.float32), n)
+    expect = f32_from_bf16_bits(base) * (2.0 ** e).astype(np.float32)
+    assert np.array_equal(f32_from_bf16_bits(moved), expect)
+
+
 def test_row_sample_is_exact():
     w = synth.custom(22, 1, 300, 2, 64, rope=False)
     q8, qs = O.quant_q(w.q)

@@ -450,6 +450,18 @@ def test_v_scale_is_applied_per_output_channel():
     assert np.array_equal(f32_from_bf16_bits(moved), expect)
 
 
+def test_batch_entries_are_independent_problems():
+    # each batch entry is its own problem (per-(b, h) means, scales and softmax):
+    # the B = 2 pipeline equals the two B = 1 pipelines stacked, bit for bit
+    w = synth.custom(23, 2, 140, 2, 64, rope=False)
+    both = O.pipeline(w.q, w.k, w.v, w.q_weight, w.k_weight, w.eps, w.rotary_dim, w.theta)
+    for b in range(2):
+        one = O.pipeline(w.q[b:b + 1], w.k[b:b + 1], w.v[b:b + 1], w.q_weight, w.k_weight,
+                         w.eps, w.rotary_dim, w.theta)
+        for key in ("q8", "q_scale", "k8", "k_scale", "k_mean", "v8t", "v_scale", "out"):
+            assert np.array_equal(both[key][b:b + 1], one[key]), (b, key)
+
+
 def test_row_sample_is_exact():
     w = synth.custom(22, 1, 300, 2, 64, rope=False)
     q8, qs = O.quant_q(w.q)

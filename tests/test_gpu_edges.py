@@ -93,6 +93,19 @@ def test_per_token_k_scales_d128(Nq, Nkv, Hq, Hkv):
     assert_out_close(host(pipe.out), out, "per-token K scales, D=128")
 
 
+def test_prep_position_offset():
+    # RoPE positions pos_offset + n ("Preparation" step 3), bit-exact against the oracle
+    w = synth.custom(25, 1, 300, 2, 128)
+    pipe = qa.Pipeline(1, 300, 300, 2, 2, 128, device=DEV)
+    pipe.run_prep(dev_bf16(w.q), dev_bf16(w.k), dev_bf16(w.q_weight), dev_bf16(w.k_weight), w.eps,
+                  w.rotary_dim, w.theta, pos_offset=777)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pipe.qp), O.prep(w.q, w.q_weight, w.eps, w.rotary_dim, w.theta,
+                                                 pos_offset=777))
+    assert np.array_equal(host(pipe.kp), O.prep(w.k, w.k_weight, w.eps, w.rotary_dim, w.theta,
+                                                 pos_offset=777))
+
+
 def test_interleaved_strided_equals_contiguous():
     # GPU-vs-GPU: the interleaved QKV buffer and contiguous copies give identical bytes
     B, N, H, D = 1, 333, 4, 128

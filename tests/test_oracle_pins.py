@@ -179,6 +179,21 @@ def test_rope_preserves_pair_norm_and_relative_position():
 
 
 # ================================================================ K mean
+def test_rope_position_offset_shifts_positions():
+    # "Preparation" step 3 with positions pos_offset + n: prep at offset p equals
+    # prep of the same rows placed at n + p with offset 0, and the explicit list
+    rng = np.random.default_rng(24)
+    n, p = 12, 1000
+    x = _bf(rng.standard_normal((1, n, 2, 128)).astype(np.float32))
+    w = _bf((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    shifted = O.prep(x, w, 1e-5, 96, pos_offset=p)
+    big = np.zeros((1, n + p, 2, 128), dtype=np.uint16)
+    big[:, p:] = x
+    assert np.array_equal(shifted, O.prep(big, w, 1e-5, 96)[:, p:])
+    assert np.array_equal(shifted, O.prep(x, w, 1e-5, 96, positions=np.arange(p, p + n)))
+    assert not np.array_equal(shifted, O.prep(x, w, 1e-5, 96))
+
+
 def test_k_mean_closed_forms():
     n = 200
     k = np.zeros((1, n, 2, 64), np.float32)

@@ -106,6 +106,20 @@ def test_prep_position_offset():
                                                  pos_offset=777))
 
 
+def test_custom_softmax_scale():
+    # qattn_fwd's sm_scale: c = FP32(log2(e) * sm_scale) instead of log2(e)/sqrt(D)
+    w = synth.make("small")
+    pipe = run_pipeline(w)
+    default = host(pipe.out).copy()
+    pipe.run_fwd(sm_scale=0.05)
+    pipe.check()
+    ref = oracle_full(w)
+    out, _, _ = O.attention(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], ref["v8t"],
+                            ref["v_scale"], w.Nkv, sm_scale=0.05)
+    assert_out_close(host(pipe.out), out, "sm_scale 0.05")
+    assert not np.array_equal(host(pipe.out), default)
+
+
 def test_interleaved_strided_equals_contiguous():
     # GPU-vs-GPU: the interleaved QKV buffer and contiguous copies give identical bytes
     B, N, H, D = 1, 333, 4, 128

@@ -106,6 +106,17 @@ def test_prep_position_offset():
                                                  pos_offset=777))
 
 
+def test_prep_without_norm_and_partial_rotary():
+    # NULL weight: no RMSNorm for that tensor (Q here), RoPE still applied; K with
+    # its norm; rotary_dim 64 of D = 128 (dims 64.. pass through)
+    w = synth.custom(26, 1, 200, 3, 128)
+    pipe = qa.Pipeline(1, 200, 200, 3, 3, 128, device=DEV)
+    pipe.run_prep(dev_bf16(w.q), dev_bf16(w.k), None, dev_bf16(w.k_weight), w.eps, 64, w.theta)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pipe.qp), O.prep(w.q, None, w.eps, 64, w.theta))
+    assert np.array_equal(host(pipe.kp), O.prep(w.k, w.k_weight, w.eps, 64, w.theta))
+
+
 def test_custom_softmax_scale():
     # qattn_fwd's sm_scale: c = FP32(log2(e) * sm_scale) instead of log2(e)/sqrt(D)
     w = synth.make("small")

@@ -14,8 +14,8 @@
 //               kind::i8 (M=128, N=64, K=32 steps; for D >= 128 the Q tile is
 //               operand A in TMEM, stored there once by the softmax warps) into
 //               TMEM S[i] as soon as the softmax warps have read S[i], then P.V
-//               as kind::f8f6f4 with P
-//               read from TMEM (M=128, N=D, K=32) accumulating into TMEM O[i]
+//               as kind::f8f6f4 with P read from TMEM (M=128, N=D, K=32)
+//               accumulating into TMEM O[i]
 //   warps 4..   D <= 128: one 128-thread softmax warpgroup per query tile;
 //               thread r owns query row r (TMEM lane r): tcgen05.ld of its 64
 //               scores, the online-softmax update, tcgen05.st of its 64 FP8
@@ -23,7 +23,8 @@
 //               row's maximum moved, after the previous P.V completed), and the
 //               final normalisation + BF16 store.  S is preloaded with the bits
 //               of 1.5 * 2^23 and QK accumulates onto them, so the scores read
-//               back as FP32 with one packed subtract per pair and no conversion.
+//               back as FP32 with one packed subtract per pair and no conversion;
+//               the reader re-preloads S and releases it to the next QK at once.
 //   warps 3..   D = 256: two warpgroups per query tile, one per half of the 64
 //               keys (and of the O columns); the two warps on the same rows swap
 //               their half-row maxima through shared memory every tile, and add

@@ -61,6 +61,14 @@ def init_dist(world: int, backend: str):
     return dist if world > 1 else None
 
 
+def percentile(values, q: float) -> float:
+    """The q-quantile (0..1) of a list by the nearest-rank rule on the sorted values."""
+    v = sorted(values)
+    if not v:
+        raise ValueError("no values")
+    return v[min(len(v) - 1, max(0, round(q * (len(v) - 1))))]
+
+
 def max_over_ranks(x: float, dist, device=None) -> float:
     """Largest value of x over all ranks (x itself with one rank)."""
     if dist is None:
@@ -304,7 +312,8 @@ def run_gpu(args):
     ms_total = t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
+    fwd_all = [a.elapsed_time(b) for a, b in fwd_events]
+    fwd_ms = statistics.mean(fwd_all)
     value = sum_over_ranks(flops, dist, dev) / (ms_step / 1e3) / 1e12
 
     # ---- end-to-end: pinned host QKV in, host output back, every step, through
@@ -362,6 +371,8 @@ def run_gpu(args):
             "dtype": "int8 QK / e4m3 PV (f32 accumulate), bf16 in/out", "data": "synthetic",
             "config": dict(workload_config(w), parallelism=f"{world} independent problems (one per GPU)"),
             "fwd_ms_per_call": fwd_ms,
+            "fwd_ms_p10": percentile(fwd_all, 0.1),
+            "fwd_ms_p90": percentile(fwd_all, 0.9),
             "fwd_tflops": achieved,
             "fwd_frac_of_spec_4500": achieved / SPEC_FP8_TFLOPS,
             "prep_quant_ms": ms_step - fwd_ms,

@@ -64,3 +64,14 @@ def test_shard_heads_partitions_every_head_once(H, world):
     assert covered == list(range(H))
     sizes = [b - a for a, b in ranges]
     assert max(sizes) - min(sizes) <= 1
+
+
+def test_percentile_nearest_rank():
+    import bench
+    vals = [5.0, 1.0, 3.0, 2.0, 4.0]
+    assert bench.percentile(vals, 0.0) == 1.0
+    assert bench.percentile(vals, 1.0) == 5.0
+    assert bench.percentile(vals, 0.5) == 3.0
+    assert bench.percentile([7.0], 0.9) == 7.0
+    ten = [float(i) for i in range(10)]
+    assert bench.percentile(ten, 0.1) == 1.0 and bench.percentile(ten, 0.9) == 8.0

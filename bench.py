@@ -2,7 +2,7 @@
 
 One step = the whole hot path on the canonical call of the "Exact Numerical
 Contract" page: B=1, N=37,810, H=56, D=128, interleaved BF16 QKV [N, 21504]:
-  qattn_prep (RMSNorm + RoPE) -> qattn_quant (K mean, INT8 Q/K, FP8 V)
+  qattn_prep_quant (RMSNorm + RoPE, K mean, INT8 Q/K, FP8 V; two HBM passes)
   -> qattn_fwd (tcgen05 INT8 QK^T, online softmax, FP8 P.V, BF16 out).
 Value = effective TFLOP/s = 4*B*H*N^2*D per step (all ranks) / step time
 (max over ranks).  Each rank runs its own independent problem (weak scaling,
@@ -35,13 +35,14 @@ WORKLOAD = {"workload": "canonical interleaved-QKV quantized attention prefill",
             "rotary_dim": 96, "causal": False,
             "l2": "inputs larger than L2 (1.63 GB QKV, 126 MB L2); no flush needed"}
 NOMINAL_FP8_OVER_BF16 = 2.0          # 4.5 / 2.25 PFLOP/s dense (nominal ratio)
-# DRAM bytes per canonical attention launch: ncu dram__bytes_read + write on the
-# B1 N16384 H32 D128 case (201.5 MB + 102.5 MB = 304.1 MB) scaled by the units
-# processed (N*H: 2117360 / 524288 = 4.0386).  Valid only for the attention kernel
-# the capture was taken on (this file's kernel as of the capture); set to None when
-# the kernel changes and re-take the capture.
-ATTN_TRAFFIC_BYTES = int((201517312 + 102539520) * 2117360 / 524288)
+# DRAM bytes per canonical attention launch: ncu dram__bytes_read + write of one
+# attention launch on the B1 N16384 H32 D128 case, scaled by the units processed
+# (N*H: 2117360 / 524288 = 4.0386).  Valid only for the attention kernel the
+# capture was taken on; None until it is re-taken after a kernel change.
+ATTN_TRAFFIC_BYTES = None
+ATTN_TRAFFIC_SOURCE = None
 SPEC_FP8_TFLOPS = 4500.0
+PROBE_MMA_MACS = 128 * 256 * 32      # multiply-adds of one probe MMA (M128 N256 K32)
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -152,6 +153,46 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def prep_quant_bytes(w) -> int:
+    """Algorithmic HBM bytes of one qattn_prep_quant call (or, for the rotated
+    variant, of qattn_quant_hadamard): every tensor read or written once per pass
+    that touches it.  Fused path: raw Q, K, V read and INT8 Q written (pass 1),
+    FP64 K sums and FP32 V maxima per 64-row block written and read back, raw K and
+    V read again and INT8 K and E4M3 V (padded to 64-row blocks) written (pass 2)."""
+    nk = -(-w.Nkv // 64)
+    q_in = 2 * w.B * w.Nq * w.Hq * w.D
+    kv_in = 2 * w.B * w.Nkv * w.Hkv * w.D
+    q8 = w.B * w.Nq * w.Hq * w.D
+    k8 = w.B * w.Nkv * w.Hkv * w.D
+    v8 = w.B * w.Hkv * w.D * 64 * nk
+    partials = 2 * 12 * w.B * nk * w.Hkv * w.D
+    if w.hadamard:   # V statistics pass, then Q, K and V quantized
+        return kv_in + 4 * w.B * nk * w.Hkv * w.D * 2 + q_in + 2 * kv_in + q8 + k8 + v8
+    return (q_in + 2 * kv_in + q8) + partials + (2 * kv_in + k8 + v8)
+
+
+def tc_probe(dev, kind: int, iters: int = 8192):
+    """The library's tensor-core peak probe (one CTA per SM, back-to-back M128 N256
+    K32 MMAs from shared memory): event-timed TFLOP/s and multiply-adds per clock
+    per SM from the in-kernel cycle count."""
+    import torch
+    import quantized_exact_attention_qattn_b200 as qa
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    cycles = torch.zeros(1, dtype=torch.int64, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    qa.qattn_tc_probe(kind, 256, n_sm, cycles, err)
+    qa.qattn_check(err)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    qa.qattn_tc_probe(kind, iters, n_sm, cycles, err)
+    e1.record()
+    qa.qattn_check(err)
+    ms = e0.elapsed_time(e1)
+    macs_clk = iters * PROBE_MMA_MACS / int(cycles.item())
+    return {"tflops": 2.0 * n_sm * iters * PROBE_MMA_MACS / (ms / 1e3) / 1e12,
+            "macs_per_clk_per_sm": macs_clk, "n_sm": n_sm, "iters": iters}
 
 
 # ------------------------------------------------------------------ workloads
@@ -271,21 +312,29 @@ def run_gpu(args):
     if w.q_weight is not None:
         qw = torch.from_numpy(w.q_weight).view(torch.bfloat16).to(dev)
         kw = torch.from_numpy(w.k_weight).view(torch.bfloat16).to(dev)
-    pipe = qa.Pipeline(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, hadamard=w.hadamard, device=dev)
+    pipe = qa.Pipeline(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, hadamard=w.hadamard,
+                       fused=not w.hadamard, rotary_dim=w.rotary_dim, device=dev)
     stream = torch.cuda.current_stream(dev)
     flops = pipe.attn_ops
 
-    def step(fwd_ev=None):
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
         if w.hadamard:
             pipe.run_quant_hadamard(q, k, v)
         else:
-            pipe.run_prep(q, k, qw, kw, w.eps, w.rotary_dim, w.theta)
-            pipe.run_quant(pipe.qp, pipe.kp, v)
-        if fwd_ev is not None:
-            fwd_ev[0].record(stream)
+            pipe.run_prep_quant(q, k, v, qw, kw, w.eps, w.theta)
+        if ev is not None:
+            ev[1].record(stream)
         pipe.run_fwd()
-        if fwd_ev is not None:
-            fwd_ev[1].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    probe = {}
+    if rank == 0 and not args.no_probe:
+        with ClockSampler(local) as pclk:
+            probe = {"i8": tc_probe(dev, 0), "e4m3": tc_probe(dev, 1)}
+        probe["clocks"] = pclk.summary()
 
     for _ in range(args.warmup):
         step()
@@ -293,7 +342,7 @@ def run_gpu(args):
     pipe.check()
 
     # ---- device-timed region
-    fwd_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    fwd_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                   for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
@@ -312,8 +361,9 @@ def run_gpu(args):
     ms_total = t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
-    fwd_all = [a.elapsed_time(b) for a, b in fwd_events]
+    fwd_all = [b.elapsed_time(c) for a, b, c in fwd_events]
     fwd_ms = statistics.mean(fwd_all)
+    pq_ms = statistics.mean([a.elapsed_time(b) for a, b, c in fwd_events])
     value = sum_over_ranks(flops, dist, dev) / (ms_step / 1e3) / 1e12
 
     # ---- end-to-end: pinned host QKV in, host output back, every step, through
@@ -357,13 +407,40 @@ def run_gpu(args):
                 peaks = json.load(f)
         except OSError:
             pass
-        if "bf16_tflops_sustained" in peaks:
+        clocks = clk.summary()
+        # burst figure when the attention kernel ran at the maximum SM clock (it does
+        # not reach the power cap), the sustained one when the clock sagged
+        at_max = (clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and
+                  clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"])
+        if "bf16_tflops" in peaks and at_max:
+            peak = peaks["bf16_tflops"] * NOMINAL_FP8_OVER_BF16
+            peak_src = ("of measured: MEASURED_PEAKS bf16 burst x nominal fp8/bf16 ratio 2 "
+                        "(SM clock at max during the timed region)")
+        elif "bf16_tflops_sustained" in peaks:
             peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP8_OVER_BF16
-            peak_src = "measured bf16 sustained x nominal fp8/bf16 ratio 2"
+            peak_src = ("of measured: MEASURED_PEAKS bf16 sustained x nominal fp8/bf16 ratio 2 "
+                        "(SM clock below max during the timed region)")
         else:
-            peak = 1400.0 * NOMINAL_FP8_OVER_BF16
-            peak_src = "fallback bf16 sustained 1.4 PFLOP/s x nominal ratio 2"
+            peak = 1590.0 * NOMINAL_FP8_OVER_BF16
+            peak_src = "of fallback: bf16 burst 1.59 PFLOP/s x nominal ratio 2"
+        hbm = peaks.get("hbm_gbs", 6650.0)
+        hbm_src = "of measured" if "hbm_gbs" in peaks else "of fallback"
         achieved = flops / (fwd_ms / 1e3) / 1e12
+        pq_bytes = prep_quant_bytes(w)
+        probe_line = None
+        if probe:
+            mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz")
+            i8_peak = 2.0 * probe["i8"]["macs_per_clk_per_sm"] * probe["i8"]["n_sm"] * mhz * 1e6 / 1e12
+            probe_line = {
+                "i8_tflops_event_timed": probe["i8"]["tflops"],
+                "e4m3_tflops_event_timed": probe["e4m3"]["tflops"],
+                "i8_macs_per_clk_per_sm": probe["i8"]["macs_per_clk_per_sm"],
+                "e4m3_macs_per_clk_per_sm": probe["e4m3"]["macs_per_clk_per_sm"],
+                "probe_clocks": probe["clocks"],
+                "i8_peak_at_attention_clock": i8_peak,
+                "frac_of_probe_peak": achieved / i8_peak,
+                "kernel": "qattn_tc_probe: one CTA per SM, back-to-back M128 N256 K32 MMAs "
+                          "from shared memory"}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -375,10 +452,17 @@ def run_gpu(args):
             "fwd_ms_p90": percentile(fwd_all, 0.9),
             "fwd_tflops": achieved,
             "fwd_frac_of_spec_4500": achieved / SPEC_FP8_TFLOPS,
-            "prep_quant_ms": ms_step - fwd_ms,
+            "prep_quant_ms": pq_ms,
+            "prep_quant": {"call": "qattn_quant_hadamard" if w.hadamard else "qattn_prep_quant",
+                           "ms": pq_ms, "algorithmic_bytes": pq_bytes,
+                           "gbs": pq_bytes / (pq_ms / 1e3) / 1e9,
+                           "frac_of_hbm": pq_bytes / (pq_ms / 1e3) / 1e9 / hbm,
+                           "hbm_gbs": hbm, "hbm_source": hbm_src},
+            "tensor_probe": probe_line,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "traffic": ATTN_TRAFFIC_BYTES if args.config == "canonical" else None,
+                         "traffic_source": ATTN_TRAFFIC_SOURCE if args.config == "canonical" else None,
                          "kernel": "attn_fwd_kernel<%d,%d,%d>" % (w.D, {64: 3, 128: 2}.get(w.D, 1),
                                                                   1 if w.hadamard else 0),
                          "peak_source": peak_src,
@@ -388,8 +472,10 @@ def run_gpu(args):
                     "call": "qattn_attention_host, %d KV heads per chunk" % (runner.chunk if runner else 0),
                     "h2d_bytes_per_step": host_qkv.numel() * 2,
                     "d2h_bytes_per_step": out_host.numel() * 2},
-            "gpu_launches": (3 if w.hadamard else 5) * args.steps,
-            "clocks": clk.summary(),
+            # rope table (when R > 0), pass 1, finalize, pass 2, attention; rotated
+            # path: V statistics (2), rotation + quant, V quant, attention
+            "gpu_launches": (5 if w.hadamard else (5 if w.rotary_dim > 0 else 4)) * args.steps,
+            "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline and args.config == "canonical":
             line["cpu_baseline"] = cpu_baseline_line(w)
@@ -408,6 +494,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-probe", action="store_true", help="skip the tensor-core peak probe")
     ap.add_argument("--e2e-chunk", type=int, default=None,
                     help="KV heads per chunk of the end-to-end call (default Hkv // 8)")
     ap.add_argument("--config", default="canonical",

@@ -114,6 +114,56 @@ qattn_status qattn_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
                          float* k_mean, uint8_t* v8t, float* v_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Same as qattn_quant with one K scale per 32-row group instead of per 64-row
+ * block: the finer grouping the page "npu plan P7" names for heads whose outliers
+ * survive ("per-32-group scales at a small byte cost").  The K arithmetic is that
+ * of qattn_quant over 32 rows (x = (float)k - k_mean, amax/127, rni_sat_s8);
+ * k_scale is FP32 [B,Hkv,ceil(Nkv/32)].  Use qattn_fwd with k_scale_mode 2.
+ * Other arguments, layouts and errors as qattn_quant. */
+qattn_status qattn_quant_k32(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                             qattn_bnhd qp, qattn_bnhd kp, qattn_bnhd v,
+                             int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                             float* k_mean, uint8_t* v8t, float* v_scale,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* V for the FP16 P.V product (page "Fused FP8 PV preparation": FP16 PV is the
+ * default, FP8 probabilities the option): v16 = fp16_rn(v) from BF16, no scale
+ * (exact wherever |v| lies in FP16's normal range), stored dim-major like the FP8
+ * V, keys contiguous: v16t FP16 [B,Hkv,D,capacity] (device), entries past Nkv
+ * written as 0.  capacity >= Nkv, a multiple of 8.
+ * Errors: NULL, SHAPE, STRIDE, UNSUPPORTED, CUDA. */
+qattn_status qattn_quant_v16(int B, int Nkv, int Hkv, int D, qattn_bnhd v, uint16_t* v16t,
+                             int capacity, void* stream);
+
+/* ---------------------------------------------------------------- prep + quant, fused
+ * qattn_prep followed by qattn_quant on the same self-attention inputs, in two
+ * passes over HBM instead of four ("Exact Numerical Contract", "Preparation"
+ * steps 1-4, "Q And K Quantization", "V And PV").  Every output is bit for bit
+ * what qattn_prep -> qattn_quant give (the prepared BF16 Q and K are the same
+ * values; they are only not stored):
+ *   pass 1  raw Q, K, V read once: Q prepared and quantized per 32-row group in
+ *           registers; K prepared and summed per 64-row block (FP64, rows
+ *           ascending); V column maxima per block
+ *   finalize  K mean (blocks ascending, FP64, / N, rounded once), V scales
+ *   pass 2  raw K, V read again: K prepared again, mean subtracted, quantized per
+ *           64-row block; V quantized to E4M3 and stored dim-major
+ * The RoPE coefficients (the same FP64 -> BF16 values as qattn_prep, positions
+ * pos_offset + n) are tabulated once per call into the workspace.
+ * Arguments
+ *   q [B,N,Hq,D], k and v [B,N,Hkv,D]   RAW strided BF16 views (device)
+ *   q_weight, k_weight, eps, rotary_dim, rope_theta, pos_offset   as qattn_prep
+ *   q8, q_scale, k8, k_scale, k_mean, v8t, v_scale   as qattn_quant (Nq = Nkv = N)
+ *   workspace   device, 256-byte aligned, >= qattn_prep_quant_workspace_bytes(...)
+ * Errors: NULL, SHAPE, STRIDE, UNSUPPORTED, WORKSPACE, CUDA. */
+size_t qattn_prep_quant_workspace_bytes(int B, int N, int Hkv, int D, int rotary_dim);
+qattn_status qattn_prep_quant(int B, int N, int Hq, int Hkv, int D,
+                              qattn_bnhd q, qattn_bnhd k, qattn_bnhd v,
+                              const uint16_t* q_weight, const uint16_t* k_weight, float eps,
+                              int rotary_dim, double rope_theta, int64_t pos_offset,
+                              int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                              float* k_mean, uint8_t* v8t, float* v_scale,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* Hadamard-rotated variant ("npu plan P7" page: rotate Q and K by the same
  * per-head Walsh-Hadamard H, store K int8 with one FP16 scale per (head, token)).
  *   x' = FWHT(x) / sqrt(D) in FP32 (Sylvester order, no sign vector; stages
@@ -131,18 +181,21 @@ qattn_status qattn_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* Same computation as qattn_quant, for callers that cannot allocate device
- * memory when they quantize (inside a CUDA-graph capture, under an allocator
- * that forbids allocation on the hot path, or in an embedder whose memory
- * manager hands out only the tensors).  The pages have no counterpart: it is
- * an interface choice of this library, not part of the method.
+ * memory when they quantize: an embedder whose memory manager owns all device
+ * memory and hands out only the tensors, or a runtime that must not allocate on
+ * its hot path because cudaMalloc / cudaFree can synchronize the device.  The
+ * pages have no counterpart: it is an interface choice of this library, not part
+ * of the method.
  * The scratch lives in one static device array of QATTN_NOALLOC_SCRATCH_BYTES
- * (16 MiB) compiled into the library; every device that uses the entry point
- * keeps it until the process exits.  Problems whose qattn_quant_workspace_bytes
- * exceeds that are refused with QATTN_ERR_WORKSPACE.  All calls share the
- * array, so calls that overlap on the GPU (other streams or threads) race:
- * serialize them.  No scratch byte needs clearing between calls.  The first
- * call on each device looks up the array's device address (cudaGetSymbolAddress)
- * and caches it; make that first call before any stream capture.
+ * (16 MiB) compiled into the library; every device on which the library's module
+ * is loaded holds it until the process exits.  Problems whose
+ * qattn_quant_workspace_bytes exceeds that are refused with QATTN_ERR_WORKSPACE.
+ * All calls share the array, so calls that overlap on the GPU (other streams or
+ * threads) race: serialize them.  No scratch byte needs clearing between calls
+ * (each call writes every byte it reads).  The first call in each CUDA context
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it under
+ * the context's unique ID; make that first call before any stream capture, and
+ * again first after a cudaDeviceReset.
  * Arguments, layouts and errors otherwise as qattn_quant. */
 #define QATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 qattn_status qattn_quant_noalloc(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
@@ -154,16 +207,22 @@ qattn_status qattn_quant_noalloc(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  * Fused attention ("INT8 QK And Score Domain", "Online Softmax", "V And PV",
  * "Finalization And Tails").  Per query row, over 64-key tiles t = 0, 1, ... in
  * order, with m = -5e6f, d = 1.0f, O = 0 initially:
- *   s_j  = ((float)S_j * (q_scale * k_scale_j)) * c, c = log2(e) * sm_scale,
- *          S = Q8 K8^T exact in INT32; keys >= Nkv get -5e6f
+ *   S_j  = Q8 K8^T exact in INT32
+ *   A_j  = (q_scale * k_scale_j) * c  (FP32), c = (float)(log2(e) * sm_scale)
+ *   s_j  = S_j * A_j (FP32); keys >= Nkv are masked (p_j = 0)
  *   mn   = max(m, max_j s_j - 8.807f); old = 2^(m - mn); d *= old; O *= old
- *   p_j  = 2^(s_j - mn); d += p_j (FP32, unquantized); P8 = e4m3_rn_satfinite(p)
- *   O   += P8 . V8 (tcgen05 FP8 MMA, FP32 accumulation in tensor memory)
- *   out  = bf16_rn(O / d * v_scale[d]), query rows < Nq only.
+ *   p_j  = 2^fma(S_j, A_j, -mn) (the exponent rounded once); d += p_j (FP32,
+ *          unquantized); P8 = e4m3_rn_satfinite(p_j)
+ *   O   += P8 . V8 (tcgen05 FP8 MMA, FP32 accumulation in tensor memory); m = mn
+ *   out  = bf16_rn(O * rcp(d) * v_scale[d]), query rows < Nq only.
+ * 2^x is ex2.approx or an FMA-pipe polynomial of equal accuracy; the sums run in
+ * FP32 in an order of the kernel's own (within the output tolerance).
  * Arguments (all device except scalars)
  *   q8, q_scale, k8, v8t, v_scale  as produced by qattn_quant / _hadamard
  *   k_scale       k_scale_mode 0: FP32 [B,Hkv,ceil(Nkv/64)];
- *                 k_scale_mode 1: FP16 [B,Hkv,Nkv] (per token)
+ *                 k_scale_mode 1: FP16 [B,Hkv,Nkv] (per token);
+ *                 k_scale_mode 2: FP32 [B,Hkv,ceil(Nkv/32)] (per 32-row group,
+ *                 qattn_quant_k32; A_j takes key j's group scale)
  *   sm_scale      softmax scale; 0 means 1/sqrt(D)
  *   out           contiguous BF16 [B,Nq,Hq,D]
  *   dev_err       one int32 (device), caller-owned; the kernel ORs error bits into
@@ -176,16 +235,74 @@ qattn_status qattn_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
                        const uint8_t* v8t, const float* v_scale, float sm_scale,
                        uint16_t* out, int* dev_err, void* stream);
 
-/* Raw INT32 score tiles S = Q8 K8^T through the same TMA + tcgen05 INT8 path as
- * qattn_fwd ("INT8 QK And Score Domain"), for bit-exact checks.
- *   tiles    int32 [n_tiles][4] = (b, h, q_tile, k_tile) (device); q_tile indexes
- *            128-row query tiles, k_tile 64-row key tiles; rows past Nq/Nkv read 0
- *   s_out    int32 [n_tiles][128][64] (device)
- * Errors: NULL, SHAPE, UNSUPPORTED, CUDA; TIMEOUT via dev_err. */
+/* The FP16 P.V control of the page "Fused FP8 PV preparation": qattn_fwd with
+ * the probabilities encoded as FP16 (P16 = fp16_rn(p), same softmax, maximum and
+ * unquantized denominator) and V as FP16 from qattn_quant_v16, multiplied by
+ * tcgen05 kind::f16 with FP32 accumulation in tensor memory; out = bf16_rn(O *
+ * rcp(d)) (no V scale).
+ *   k8, k_scale  as qattn_fwd, but the rows (and per-token scales) of one (batch,
+ *                KV head) are kv_capacity apart: k8 [B,Hkv,kv_capacity,D],
+ *                k_scale mode 0 [B,Hkv,ceil(cap/64)], mode 1 [B,Hkv,cap], mode 2
+ *                [B,Hkv,ceil(cap/32)]; only the first Nkv keys are used
+ *   v16t         FP16 [B,Hkv,D,kv_capacity] (device)
+ *   kv_capacity  >= Nkv, a multiple of 8 (Nkv rounded up for a plain problem;
+ *                the allocated length of a key cache)
+ * Errors: as qattn_fwd; SHAPE for kv_capacity. */
+qattn_status qattn_fwd_pv16(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                            const int8_t* q8, const float* q_scale,
+                            const int8_t* k8, const void* k_scale, int k_scale_mode,
+                            const uint16_t* v16t, int kv_capacity, float sm_scale,
+                            uint16_t* out, int* dev_err, void* stream);
+
+/* INT32 score tiles S = Q8 K8^T exactly as the attention mainloop computes them
+ * ("INT8 QK And Score Domain"), for bit-exact checks of the path qattn_fwd runs.
+ * This launches qattn_fwd's own kernel on the whole problem (same operands, same
+ * TMA copies, same tcgen05 kind::i8 MMAs with Q read from tensor memory at D 128
+ * and 256 and from shared memory at D 64, same 1.5*2^23 preload at D <= 128 and
+ * integer-to-float conversion at D 256), built with one addition: when the softmax
+ * warps have recovered the scores of a requested tile from tensor memory, they
+ * also copy them out.  `out` receives the attention output as from qattn_fwd.
+ *   tiles    int32 [n_tiles][4] = (b, h, q_tile, k_tile) (device, 16-byte
+ *            aligned); q_tile indexes 128-row query tiles, k_tile 64-key tiles.
+ *            Entries naming no tile of the problem leave their slot untouched.
+ *   s_out    int32 [n_tiles][128][64] (device, 16-byte aligned); rows past Nq and
+ *            keys past Nkv read as 0 (zero rows of the operands)
+ *   n_tiles  1 .. QATTN_SCORES_MAX_TILES
+ * Other arguments and errors as qattn_fwd; also NULL (tiles, s_out), SHAPE
+ * (n_tiles), STRIDE (alignment).  A debugging aid: slower than qattn_fwd. */
+#define QATTN_SCORES_MAX_TILES 65536
 qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
-                          const int8_t* q8, const int8_t* k8,
+                          const int8_t* q8, const float* q_scale,
+                          const int8_t* k8, const void* k_scale, int k_scale_mode,
+                          const uint8_t* v8t, const float* v_scale, float sm_scale,
                           const int32_t* tiles, int n_tiles, int32_t* s_out,
-                          int* dev_err, void* stream);
+                          uint16_t* out, int* dev_err, void* stream);
+
+/* ---------------------------------------------------------------- key cache
+ * Chunked prefill into a persistent rotated int8 key cache (page "npu plan P7:
+ * int8 KV with per-head Hadamard rotation": prefill in 1024/2048-token chunks
+ * writes the KV in the contract the decode path reads; the design note's first
+ * variant keeps K int8, rotated, with a per-token scale sidecar, and V in 16
+ * bits; rotating Q by the same H leaves the scores unchanged, so K is never
+ * un-rotated).  One (batch, KV head) plane of the cache holds `capacity` keys:
+ *   k8_cache      int8 [B,Hkv,capacity,D]
+ *   k_scale_cache FP16 [B,Hkv,capacity]     (per-token scales, as qattn_quant_hadamard)
+ *   v16_cache     FP16 [B,Hkv,D,capacity]   (dim-major, as qattn_quant_v16)
+ * qattn_kcache_append writes the n_new keys of one chunk at positions key0 ..
+ * key0+n_new-1: K' = FWHT(k)/sqrt(D) then INT8 with one FP16 scale per token
+ * (the arithmetic of qattn_quant_hadamard's K), V as FP16; the V slots up to
+ * key0 + n_new rounded up to 8 are written (the padding as 0), nothing else.
+ * key0 and capacity are multiples of 8, key0 + n_new rounded up to 8 <= capacity,
+ * D in {64, 256}; k and v are the chunk's raw BF16 [B,n_new,Hkv,D] (device).
+ * A query chunk then uses qattn_quant_q_hadamard (Q' = FWHT(q)/sqrt(D), INT8 per
+ * 32-row group) and qattn_fwd_pv16 with Nkv = key0 + n_new, k_scale_mode 1 and
+ * kv_capacity = capacity: attention over every key cached so far.
+ * Errors: NULL, SHAPE, STRIDE, UNSUPPORTED, CUDA. */
+qattn_status qattn_kcache_append(int B, int Hkv, int D, int n_new, int key0, int capacity,
+                                 qattn_bnhd k, qattn_bnhd v, int8_t* k8_cache,
+                                 uint16_t* k_scale_cache, uint16_t* v16_cache, void* stream);
+qattn_status qattn_quant_q_hadamard(int B, int Nq, int Hq, int D, qattn_bnhd q, int8_t* q8,
+                                    float* q_scale, void* stream);
 
 /* ---------------------------------------------------------------- host to host
  * The whole path for inputs and output in HOST memory, overlapping PCIe with
@@ -194,7 +311,7 @@ qattn_status qattn_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  * softmax), so this entry point cuts the KV heads into chunks of
  * kv_heads_per_chunk (each with its Hq/Hkv query heads) and streams them through
  * two device buffer sets in `workspace`: chunk c's Q/K/V go host -> device on
- * h2d_stream while chunk c-1 computes on its set's stream (qattn_prep -> qattn_quant ->
+ * h2d_stream while chunk c-1 computes on its set's stream (qattn_prep_quant ->
  * qattn_fwd, or qattn_quant_hadamard -> qattn_fwd with k_scale_mode 1) and chunk
  * c-2's output goes device -> host on d2h_stream.  The result is the same as
  * those entry points give on the whole problem, bit for bit.  The pages have no

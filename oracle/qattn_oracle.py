@@ -245,6 +245,46 @@ def quant_v(v_bits: np.ndarray):
     return v8t, v_scale
 
 
+def quant_k32(kp_bits: np.ndarray, mean: np.ndarray):
+    """K with one INT8 scale per 32-row group (the finer grouping the page "npu
+    plan P7" names for outlier heads: "per-32-group scales at a small byte
+    cost").  Reading: the same arithmetic as ``quant_k`` ("Q And K Quantization":
+    x = (f32)k - mean, amax/127, rint_sat) over 32 rows instead of 64; tail rows
+    take no part.  Returns k8 int8 [B,H,N,D] and k_scale FP32 [B,H,ceil(N/32)].
+    """
+    k = f32_from_bf16_bits(kp_bits).transpose(0, 2, 1, 3)      # [B,H,N,D]
+    x = (k - mean[:, :, None, :].astype(F32)).astype(F32)
+    b, h, n, d = x.shape
+    ng = ceil_div(n, 32)
+    xpad = np.zeros((b, h, ng * 32, d), dtype=F32)
+    xpad[:, :, :n] = x
+    valid = np.zeros((b, h, ng * 32, d), dtype=bool)
+    valid[:, :, :n] = True
+    amax = np.max(np.where(valid, np.abs(xpad), F32(0)).reshape(b, h, ng, 32, d), axis=(3, 4))
+    amax = np.maximum(AMAX_FLOOR, amax).astype(F32)
+    scale = (amax / F32(127.0)).astype(F32)
+    f = (F32(127.0) / amax).astype(F32)
+    t = (xpad.reshape(b, h, ng, 32, d) * f[..., None, None]).astype(F32)
+    k8 = np.clip(np.rint(t), -128, 127).astype(np.int8).reshape(b, h, ng * 32, d)[:, :, :n]
+    return np.ascontiguousarray(k8), scale
+
+
+def quant_v16(v_bits: np.ndarray, capacity: int | None = None):
+    """V for the FP16 P.V variant (page "Fused FP8 PV preparation": FP16 PV is the
+    default, FP8 probabilities the option).  Reading: V is converted from BF16 to
+    FP16 round-to-nearest-even with no scale (exact wherever |v| lies in FP16's
+    normal range, 2^-14 .. 65504) and stored dim-major like the FP8 V, keys
+    contiguous: uint16 FP16 bits [B,H,D,capacity] (capacity >= N, default N
+    rounded up to 8); entries past N are 0.
+    """
+    v = f32_from_bf16_bits(v_bits)                              # [B,N,H,D]
+    b, n, h, d = v.shape
+    cap = capacity if capacity is not None else 8 * ceil_div(n, 8)
+    out = np.zeros((b, h, d, cap), dtype=np.uint16)
+    out[:, :, :, :n] = f16_bits_from_f32(v).transpose(0, 2, 3, 1)
+    return out
+
+
 # ============================================================ Hadamard variant
 def fwht(x: np.ndarray) -> np.ndarray:
     """Unnormalized Walsh-Hadamard transform along the last axis, FP32.
@@ -286,20 +326,67 @@ def quant_hadamard(q_bits, k_bits, v_bits):
     Returns q8 [B,Hq,Nq,D], q_scale [B,Hq,G], k8 [B,Hkv,Nkv,D],
     k_scale_f16 uint16 [B,Hkv,Nkv], v8t, v_scale.
     """
-    qr = hadamard_rotate(q_bits).transpose(0, 2, 1, 3)           # [B,H,N,D]
-    b, h, n, d = qr.shape
-    g_total = 4 * ceil_div(n, Q_ROWS_PER_CTA)
-    qpad = np.zeros((b, h, g_total * Q_ROWS_PER_SCALE, d), dtype=F32)
-    qpad[:, :, :n] = qr
-    q8, q_scale = quant_int8(qpad.reshape(b, h, g_total, Q_ROWS_PER_SCALE, d), (3, 4))
-    q8 = np.ascontiguousarray(q8.reshape(b, h, -1, d)[:, :, :n])
+    q8, q_scale = quant_q_rotated(q_bits)
+    k8, k_scale_f16 = quant_k_rotated(k_bits)
+    v8t, v_scale = quant_v(v_bits)
+    return q8, q_scale.astype(F32), k8, k_scale_f16, v8t, v_scale
+
+
+def quant_k_rotated(k_bits):
+    """K' = K H/sqrt(D), INT8 with one FP16 scale per (batch, head, token) (the K
+    half of ``quant_hadamard``): amax = max(1e-7f, max|k'|), scale fp16_rn(amax/127),
+    q8 = rint_sat(k' * (127.0f/amax)).  Returns k8 [B,H,N,D], scales uint16 [B,H,N]."""
     kr = hadamard_rotate(k_bits).transpose(0, 2, 1, 3)           # [B,Hkv,N,D]
     amax = np.maximum(AMAX_FLOOR, np.max(np.abs(kr), axis=3, keepdims=True)).astype(F32)
     f = (F32(127.0) / amax).astype(F32)
     k8 = np.clip(np.rint((kr * f).astype(F32)), -128, 127).astype(np.int8)
     k_scale_f16 = f16_bits_from_f32((amax / F32(127.0)).astype(F32))[..., 0]
-    v8t, v_scale = quant_v(v_bits)
-    return q8, q_scale.astype(F32), k8, k_scale_f16, v8t, v_scale
+    return k8, k_scale_f16
+
+
+def quant_q_rotated(q_bits):
+    """Q' = Q H/sqrt(D), INT8 per 32-row group (the Q half of ``quant_hadamard``)."""
+    qr = hadamard_rotate(q_bits).transpose(0, 2, 1, 3)
+    b, h, n, d = qr.shape
+    g_total = 4 * ceil_div(n, Q_ROWS_PER_CTA)
+    qpad = np.zeros((b, h, g_total * Q_ROWS_PER_SCALE, d), dtype=F32)
+    qpad[:, :, :n] = qr
+    q8, q_scale = quant_int8(qpad.reshape(b, h, g_total, Q_ROWS_PER_SCALE, d), (3, 4))
+    return np.ascontiguousarray(q8.reshape(b, h, -1, d)[:, :, :n]), q_scale.astype(F32)
+
+
+# ============================================================ key cache (chunked prefill)
+def kcache_new(b: int, h: int, d: int, capacity: int) -> dict:
+    """An empty rotated int8 key cache (page "npu plan P7": int8 K rotated by a
+    per-head Hadamard with a per-token scale sidecar, V kept in 16 bits), room for
+    ``capacity`` keys per (batch, head)."""
+    return dict(k8=np.zeros((b, h, capacity, d), np.int8),
+                k_scale=np.zeros((b, h, capacity), np.uint16),
+                v16=np.zeros((b, h, d, capacity), np.uint16), n=0)
+
+
+def kcache_append(cache: dict, k_bits, v_bits) -> dict:
+    """Write one prefill chunk's keys after those already cached: K rows through
+    ``quant_k_rotated`` (each token on its own, so a chunk's codes do not depend
+    on the other chunks), V through ``quant_v16``; the cache grows by the chunk."""
+    n0, n = cache["n"], k_bits.shape[1]
+    k8, ks = quant_k_rotated(k_bits)
+    cache["k8"][:, :, n0:n0 + n] = k8
+    cache["k_scale"][:, :, n0:n0 + n] = ks
+    cache["v16"][:, :, :, n0:n0 + n] = quant_v16(v_bits, n)
+    cache["n"] = n0 + n
+    return cache
+
+
+def kcache_attend(cache: dict, q_bits, rows=None):
+    """A query chunk against every cached key: Q rotated and quantized
+    (``quant_q_rotated``), then ``attention`` with per-token K scales and the
+    FP16 P.V product (V is FP16 in the cache)."""
+    n = cache["n"]
+    q8, qs = quant_q_rotated(q_bits)
+    out, _, _ = attention(q8, qs, cache["k8"][:, :, :n], cache["k_scale"][:, :, :n],
+                          cache["v16"][..., :n], None, n, k_scale_mode=1, rows=rows, pv="fp16")
+    return out
 
 
 # ============================================================ scores
@@ -321,7 +408,7 @@ def score_constant(d: int, sm_scale: float = 0.0) -> np.float32:
 
 
 def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
-              k_scale_mode: int = 0, sm_scale: float = 0.0, rows=None):
+              k_scale_mode: int = 0, sm_scale: float = 0.0, rows=None, pv: str = "fp8"):
     """Online base-2 softmax attention over 64-key tiles, BF16 output.
 
     Follows "Online Softmax", "V And PV" and "Finalization And Tails":
@@ -346,9 +433,17 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
       m     = mn
     out = bf16_rn((f32)(RO / d) * v_scale)      (reading: exact division)
 
+    pv="fp16" is the FP16 P.V control of the page "Fused FP8 PV preparation"
+    (softmax, maximum and denominator unchanged, only the probability encoding
+    and V differ).  Reading: P16_j = fp16_rn(p_j), RO += sum_j P16_j * V16[j, :]
+    (exact tile sum) with V16 from ``quant_v16`` (no V scale), and
+    out = bf16_rn((f32)(RO / d)).
+
     Shapes: q8 [B,Hq,Nq,D], q_scale [B,Hq,G], k8 [B,Hkv,Nkv,D], k_scale
-    [B,Hkv,nK] FP32 (mode 0) or FP16 bits [B,Hkv,Nkv] (mode 1, per token),
-    v8t [B,Hkv,D,>=64*nK] E4M3 bits, v_scale [B,Hkv,D].  GQA: query head h
+    [B,Hkv,nK] FP32 (mode 0), FP16 bits [B,Hkv,Nkv] (mode 1, per token) or
+    FP32 [B,Hkv,ceil(Nkv/32)] (mode 2, per 32-row group: A_j uses the scale of
+    key j's group), v8t [B,Hkv,D,>=64*nK] E4M3 bits, v_scale [B,Hkv,D]; for
+    pv="fp16" v8t holds the FP16 bits of ``quant_v16`` and v_scale is unused.  GQA: query head h
     reads KV head h // (Hq/Hkv).  ``rows`` optionally restricts the query
     rows (independent of one another, so a sample is exact).
     Returns (out bf16 bits [B,len(rows),Hq,D], final m, final d).
@@ -366,7 +461,12 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
     m = np.full((b, hq, nr), M_INIT, dtype=F32)
     den = np.ones((b, hq, nr), dtype=F32)
     ro = np.zeros((b, hq, nr, d), dtype=np.float64)
-    v8 = f32_from_e4m3_bits(v8t).astype(np.float64)                  # [B,Hkv,D,Np]
+    if pv == "fp8":
+        vv = f32_from_e4m3_bits(v8t).astype(np.float64)              # [B,Hkv,D,Np]
+    elif pv == "fp16":
+        vv = f32_from_f16_bits(v8t).astype(np.float64)
+    else:
+        raise ValueError(pv)
     for t in range(nk):
         j0, j1 = t * KV_TILE, min(n_kv, (t + 1) * KV_TILE)
         kt = k8[:, kvh, j0:j1].astype(np.float64)                    # [B,Hq,w,D]
@@ -376,7 +476,10 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
             ks = k_scale[:, kvh, t].astype(F32)                      # [B,Hq]
             a = ((qs * ks[:, :, None]).astype(F32) * c).astype(F32)[..., None]   # [B,Hq,R,1]
         else:
-            ks = f32_from_f16_bits(k_scale[:, kvh, j0:j1])           # [B,Hq,w]
+            if k_scale_mode == 1:
+                ks = f32_from_f16_bits(k_scale[:, kvh, j0:j1])       # [B,Hq,w]
+            else:
+                ks = k_scale[:, kvh][:, :, np.arange(j0, j1) // 32].astype(F32)
             a = ((qs[..., None] * ks[:, :, None, :]).astype(F32) * c).astype(F32)  # [B,Hq,R,w]
         s = (sf * a).astype(F32)
         w = j1 - j0
@@ -396,12 +499,17 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
             p = np.concatenate([p, np.zeros(p.shape[:-1] + (KV_TILE - w,), F32)], axis=-1)
         for j in range(KV_TILE):
             den = (den + p[..., j]).astype(F32)
-        p8 = e4m3_value_from_f32(p)[..., : j1 - j0]                   # exact values
-        vt = np.swapaxes(v8[:, kvh, :, j0:j1], -1, -2)              # [B,Hq,w,D]
-        ro = ro + np.matmul(p8, vt)
+        if pv == "fp8":
+            pq = e4m3_value_from_f32(p)[..., : j1 - j0]               # exact values
+        else:
+            pq = f32_from_f16_bits(f16_bits_from_f32(p[..., : j1 - j0]))
+        vt = np.swapaxes(vv[:, kvh, :, j0:j1], -1, -2)              # [B,Hq,w,D]
+        ro = ro + np.matmul(pq.astype(np.float64), vt)
         m = mn
-    vs = v_scale[:, kvh].astype(F32)[:, :, None, :]
-    o = ((ro / den.astype(np.float64)[..., None]).astype(F32) * vs).astype(F32)
+    o = (ro / den.astype(np.float64)[..., None]).astype(F32)
+    if pv == "fp8":
+        vs = v_scale[:, kvh].astype(F32)[:, :, None, :]
+        o = (o * vs).astype(F32)
     out = bf16_bits_from_f32(o).transpose(0, 2, 1, 3)                 # [B,R,Hq,D]
     return np.ascontiguousarray(out), m, den
 

@@ -11,10 +11,16 @@ import math
 
 from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_attention_host,  # noqa: F401
                    qattn_check, qattn_debug_stall_kv_tile, qattn_fwd, qattn_host_workspace_bytes,
-                   qattn_prep, qattn_quant, qattn_quant_hadamard, qattn_quant_noalloc,
-                   qattn_quant_workspace_bytes, qattn_scores, qattn_version)
+                   qattn_prep, qattn_prep_quant, qattn_prep_quant_workspace_bytes, qattn_quant,
+                   qattn_quant_hadamard, qattn_quant_noalloc, qattn_quant_workspace_bytes,
+                   qattn_quant_k32, qattn_quant_v16, qattn_fwd_pv16, qattn_kcache_append,
+                   qattn_quant_q_hadamard,
+                   qattn_scores, qattn_tc_probe, qattn_version)
 
-__all__ = ["Pipeline", "HostRunner", "default_kv_heads_per_chunk", "QAttnError", "qattn_prep", "qattn_quant",
+__all__ = ["Pipeline", "HostRunner", "default_kv_heads_per_chunk", "QAttnError", "qattn_prep",
+           "qattn_prep_quant", "qattn_prep_quant_workspace_bytes", "qattn_tc_probe", "qattn_quant",
+           "qattn_quant_k32", "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append",
+           "qattn_quant_q_hadamard", "KCache",
            "qattn_quant_noalloc", "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
            "qattn_host_workspace_bytes", "qattn_attention_host",
@@ -27,19 +33,25 @@ def _cdiv(a, b):
 
 class Pipeline:
     """Device buffers for one problem size plus the call sequence
-    prep -> quant -> fwd (or quant_hadamard -> fwd) through the C ABI.
+    prep -> quant -> fwd (or quant_hadamard -> fwd) through the C ABI; with
+    ``fused=True`` the first two are one qattn_prep_quant call (same outputs bit
+    for bit, no prepared BF16 Q/K stored, rotary_dim fixed at construction).
 
     Buffers are allocated once (PyTorch caching allocator) and reused by every
     ``run``; nothing is computed outside the library's kernels.
     """
 
-    def __init__(self, B, Nq, Nkv, Hq, Hkv, D, *, hadamard=False, prep=True, device="cuda"):
+    def __init__(self, B, Nq, Nkv, Hq, Hkv, D, *, hadamard=False, prep=True, fused=False,
+                 rotary_dim=0, device="cuda"):
         import torch
         self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D = B, Nq, Nkv, Hq, Hkv, D
         self.hadamard, self.prep = hadamard, prep and not hadamard
+        self.fused = fused and self.prep
+        if self.fused and Nq != Nkv:
+            raise ValueError("the fused prep + quant path works on self-attention inputs")
         nq, nk = _cdiv(Nq, 128), _cdiv(Nkv, 64)
         e = dict(device=device)
-        if self.prep:
+        if self.prep and not self.fused:
             self.qp = torch.empty((B, Nq, Hq, D), dtype=torch.bfloat16, **e)
             self.kp = torch.empty((B, Nkv, Hkv, D), dtype=torch.bfloat16, **e)
         self.q8 = torch.empty((B, Hq, Nq, D), dtype=torch.int8, **e)
@@ -53,7 +65,11 @@ class Pipeline:
         self.v8t = torch.empty((B, Hkv, D, 64 * nk), dtype=torch.uint8, **e)
         self.v_scale = torch.empty((B, Hkv, D), dtype=torch.float32, **e)
         self.out = torch.empty((B, Nq, Hq, D), dtype=torch.bfloat16, **e)
-        self.ws = torch.empty(qattn_quant_workspace_bytes(B, Nkv, Hkv, D), dtype=torch.uint8, **e)
+        ws = qattn_quant_workspace_bytes(B, Nkv, Hkv, D)
+        if self.fused:
+            self.rotary_dim = rotary_dim
+            ws = qattn_prep_quant_workspace_bytes(B, Nkv, Hkv, D, rotary_dim)
+        self.ws = torch.empty(ws, dtype=torch.uint8, **e)
         self.dev_err = torch.zeros(1, dtype=torch.int32, **e)
 
     # --------------------------------------------------------------- steps
@@ -62,6 +78,12 @@ class Pipeline:
         assert self.Nq == self.Nkv, "prep works on self-attention inputs"
         qattn_prep(self.B, self.Nq, self.Hq, self.Hkv, self.D, q, k, q_weight, k_weight, eps,
                    rotary_dim, theta, pos_offset, self.qp, self.kp, stream)
+
+    def run_prep_quant(self, q, k, v, q_weight, k_weight, eps, theta=10000.0, pos_offset=0,
+                       stream=None):
+        qattn_prep_quant(self.B, self.Nq, self.Hq, self.Hkv, self.D, q, k, v, q_weight, k_weight,
+                         eps, self.rotary_dim, theta, pos_offset, self.q8, self.q_scale, self.k8,
+                         self.k_scale, self.k_mean, self.v8t, self.v_scale, self.ws, stream=stream)
 
     def run_quant(self, qp, kp, v, stream=None):
         qattn_quant(self.B, self.Nq, self.Nkv, self.Hq, self.Hkv, self.D, qp, kp, v, self.q8,
@@ -83,6 +105,10 @@ class Pipeline:
         """The whole hot path on strided BF16 [B, N, H, D] views q, k, v."""
         if self.hadamard:
             self.run_quant_hadamard(q, k, v, stream)
+        elif self.fused:
+            if rotary_dim != self.rotary_dim:
+                raise ValueError("rotary_dim differs from the one the workspace was sized for")
+            self.run_prep_quant(q, k, v, q_weight, k_weight, eps, theta, pos_offset, stream)
         elif self.prep:
             self.run_prep(q, k, q_weight, k_weight, eps, rotary_dim, theta, pos_offset, stream)
             self.run_quant(self.qp, self.kp, v, stream)
@@ -97,6 +123,55 @@ class Pipeline:
     @property
     def attn_ops(self) -> float:
         return 4.0 * self.B * self.Hq * self.Nq * self.Nkv * self.D
+
+
+class KCache:
+    """A persistent rotated int8 key cache for chunked prefill (page "npu plan
+    P7"): int8 K' = FWHT(k)/sqrt(D) with one FP16 scale per token, FP16 V, room
+    for ``capacity`` keys per (batch, KV head).  ``append`` writes one chunk's
+    keys after those already cached; ``attend`` runs a query chunk against every
+    key cached so far.  All arithmetic is in the library's kernels."""
+
+    def __init__(self, B, Hkv, D, capacity, device="cuda"):
+        import torch
+        if capacity % 8:
+            raise ValueError("capacity must be a multiple of 8")
+        self.B, self.Hkv, self.D, self.capacity = B, Hkv, D, capacity
+        e = dict(device=device)
+        self.k8 = torch.zeros((B, Hkv, capacity, D), dtype=torch.int8, **e)
+        self.k_scale = torch.zeros((B, Hkv, capacity), dtype=torch.float16, **e)
+        self.v16 = torch.zeros((B, Hkv, D, capacity), dtype=torch.float16, **e)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, **e)
+        self.n = 0
+
+    def append(self, k, v, stream=None):
+        """k, v: raw BF16 [B, n_new, Hkv, D] views of the next chunk's keys.  The
+        cache grows by n_new rounded up to a multiple of 8 (padding keys are never
+        attended: only the first ``n`` keys are)."""
+        n_new = k.shape[1]
+        if self.n % 8:
+            raise ValueError("only the last chunk may have a length that is not a multiple of 8")
+        qattn_kcache_append(self.B, self.Hkv, self.D, n_new, self.n, self.capacity, k, v, self.k8,
+                            self.k_scale, self.v16, stream)
+        self.n += n_new
+
+    def attend(self, q, out=None, sm_scale=0.0, stream=None):
+        """q: raw BF16 [B, Nq, Hq, D] query chunk (rotated and quantized here);
+        returns BF16 [B, Nq, Hq, D] attention over the cached keys."""
+        import torch
+        B, Nq, Hq, D = q.shape
+        e = dict(device=self.k8.device)
+        q8 = torch.empty((B, Hq, Nq, D), dtype=torch.int8, **e)
+        qs = torch.empty((B, Hq, 4 * _cdiv(Nq, 128)), dtype=torch.float32, **e)
+        qattn_quant_q_hadamard(B, Nq, Hq, D, q, q8, qs, stream)
+        if out is None:
+            out = torch.empty((B, Nq, Hq, D), dtype=torch.bfloat16, **e)
+        qattn_fwd_pv16(B, Nq, self.n, Hq, self.Hkv, D, q8, qs, self.k8, self.k_scale, 1, self.v16,
+                       self.capacity, sm_scale, out, self.dev_err, stream)
+        return out
+
+    def check(self, stream=None):
+        qattn_check(self.dev_err, stream)
 
 
 def default_kv_heads_per_chunk(B, Nq, Nkv, Hq, Hkv, D) -> int:

@@ -20,9 +20,13 @@ QATTN_STATUS = {0: "QATTN_OK", 1: "QATTN_ERR_NULL", 2: "QATTN_ERR_SHAPE", 3: "QA
                 7: "QATTN_ERR_TIMEOUT"}
 
 EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_noalloc",
+            "qattn_prep_quant_workspace_bytes", "qattn_prep_quant", "qattn_quant_k32",
+            "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append", "qattn_quant_q_hadamard",
             "qattn_quant_hadamard",
             "qattn_fwd", "qattn_scores", "qattn_host_workspace_bytes", "qattn_attention_host",
             "qattn_check", "qattn_debug_stall_kv_tile", "qattn_last_error", "qattn_version")
+# measurement aid, declared in include/qattn_probe.h
+EXPORTED_PROBE = ("qattn_tc_probe",)
 
 
 class QAttnError(RuntimeError):
@@ -56,22 +60,36 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_quant_workspace_bytes.restype = sz
     lib.qattn_quant.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp, vp, vp,
                                 vp, sz, vp]
+    lib.qattn_prep_quant_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.qattn_prep_quant_workspace_bytes.restype = sz
+    lib.qattn_prep_quant.argtypes = [i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, f32, i, f64, i64, vp,
+                                     vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.qattn_quant_k32.argtypes = lib.qattn_quant.argtypes
+    lib.qattn_quant_v16.argtypes = [i, i, i, i, BNHD, vp, i, vp]
+    lib.qattn_fwd_pv16.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, i, f32, vp, vp, vp]
+    lib.qattn_kcache_append.argtypes = [i, i, i, i, i, i, BNHD, BNHD, vp, vp, vp, vp]
+    lib.qattn_quant_q_hadamard.argtypes = [i, i, i, i, BNHD, vp, vp, vp]
     lib.qattn_quant_noalloc.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
                                         vp, vp, vp]
     lib.qattn_quant_hadamard.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
                                          vp, vp, sz, vp]
     lib.qattn_fwd.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, vp, vp]
-    lib.qattn_scores.argtypes = [i, i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
+    lib.qattn_scores.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, i, vp, vp,
+                                 vp, vp]
     lib.qattn_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
     lib.qattn_host_workspace_bytes.restype = sz
     lib.qattn_attention_host.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, f32, i, f64,
                                          i, f32, vp, i, vp, sz, vp, vp, vp, vp, vp]
     lib.qattn_check.argtypes = [vp, vp]
+    lib.qattn_tc_probe.argtypes = [i, i, i, vp, vp, vp]
     lib.qattn_debug_stall_kv_tile.argtypes = [i]
     lib.qattn_last_error.restype = ctypes.c_char_p
     lib.qattn_version.restype = ctypes.c_char_p
-    for name in ("qattn_prep", "qattn_quant", "qattn_quant_noalloc", "qattn_quant_hadamard", "qattn_fwd",
-                 "qattn_scores", "qattn_attention_host", "qattn_check", "qattn_debug_stall_kv_tile"):
+    for name in ("qattn_prep", "qattn_prep_quant", "qattn_quant", "qattn_quant_noalloc",
+                 "qattn_quant_k32", "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append",
+                 "qattn_quant_q_hadamard", "qattn_quant_hadamard", "qattn_fwd",
+                 "qattn_scores", "qattn_attention_host", "qattn_check", "qattn_debug_stall_kv_tile",
+                 "qattn_tc_probe"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -122,6 +140,54 @@ def qattn_quant(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_m
                               _ptr(v_scale), _ptr(workspace), nbytes, _stream(stream)))
 
 
+def qattn_prep_quant_workspace_bytes(B, N, Hkv, D, rotary_dim) -> int:
+    return int(load().qattn_prep_quant_workspace_bytes(B, N, Hkv, D, rotary_dim))
+
+
+def qattn_prep_quant(B, N, Hq, Hkv, D, q, k, v, q_weight, k_weight, eps, rotary_dim, rope_theta,
+                     pos_offset, q8, q_scale, k8, k_scale, k_mean, v8t, v_scale, workspace,
+                     workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().qattn_prep_quant(B, N, Hq, Hkv, D, bnhd(q), bnhd(k), bnhd(v), _ptr(q_weight),
+                                   _ptr(k_weight), eps, rotary_dim, rope_theta, pos_offset,
+                                   _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(k_mean),
+                                   _ptr(v8t), _ptr(v_scale), _ptr(workspace), nbytes,
+                                   _stream(stream)))
+
+
+def qattn_quant_k32(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_mean, v8t,
+                    v_scale, workspace, workspace_bytes=None, stream=None):
+    """qattn_quant with one K scale per 32-row group (k_scale [B,Hkv,ceil(Nkv/32)])."""
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().qattn_quant_k32(B, Nq, Nkv, Hq, Hkv, D, bnhd(qp), bnhd(kp), bnhd(v), _ptr(q8),
+                                  _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(k_mean), _ptr(v8t),
+                                  _ptr(v_scale), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def qattn_quant_v16(B, Nkv, Hkv, D, v, v16t, capacity, stream=None):
+    _check(load().qattn_quant_v16(B, Nkv, Hkv, D, bnhd(v), _ptr(v16t), int(capacity),
+                                  _stream(stream)))
+
+
+def qattn_fwd_pv16(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v16t,
+                   kv_capacity, sm_scale, out, dev_err, stream=None):
+    _check(load().qattn_fwd_pv16(B, Nq, Nkv, Hq, Hkv, D, _ptr(q8), _ptr(q_scale), _ptr(k8),
+                                 _ptr(k_scale), k_scale_mode, _ptr(v16t), int(kv_capacity),
+                                 sm_scale, _ptr(out), _ptr(dev_err), _stream(stream)))
+
+
+def qattn_kcache_append(B, Hkv, D, n_new, key0, capacity, k, v, k8_cache, k_scale_cache, v16_cache,
+                        stream=None):
+    _check(load().qattn_kcache_append(B, Hkv, D, n_new, key0, capacity, bnhd(k), bnhd(v),
+                                      _ptr(k8_cache), _ptr(k_scale_cache), _ptr(v16_cache),
+                                      _stream(stream)))
+
+
+def qattn_quant_q_hadamard(B, Nq, Hq, D, q, q8, q_scale, stream=None):
+    _check(load().qattn_quant_q_hadamard(B, Nq, Hq, D, bnhd(q), _ptr(q8), _ptr(q_scale),
+                                         _stream(stream)))
+
+
 def qattn_quant_noalloc(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_mean, v8t,
                         v_scale, stream=None):
     """qattn_quant on the library's static scratch (no workspace argument)."""
@@ -146,9 +212,12 @@ def qattn_fwd(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v8
                             _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
-def qattn_scores(B, Nq, Nkv, Hq, Hkv, D, q8, k8, tiles, n_tiles, s_out, dev_err, stream=None):
-    _check(load().qattn_scores(B, Nq, Nkv, Hq, Hkv, D, _ptr(q8), _ptr(k8), _ptr(tiles), n_tiles,
-                               _ptr(s_out), _ptr(dev_err), _stream(stream)))
+def qattn_scores(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v8t, v_scale,
+                 sm_scale, tiles, n_tiles, s_out, out, dev_err, stream=None):
+    _check(load().qattn_scores(B, Nq, Nkv, Hq, Hkv, D, _ptr(q8), _ptr(q_scale), _ptr(k8),
+                               _ptr(k_scale), k_scale_mode, _ptr(v8t), _ptr(v_scale), sm_scale,
+                               _ptr(tiles), n_tiles, _ptr(s_out), _ptr(out), _ptr(dev_err),
+                               _stream(stream)))
 
 
 def qattn_host_workspace_bytes(B, Nq, Nkv, Hq, Hkv, D, kv_heads_per_chunk) -> int:
@@ -168,6 +237,12 @@ def qattn_attention_host(B, Nq, Nkv, Hq, Hkv, D, q, k, v, q_weight, k_weight, ep
                                        int(hadamard), sm_scale, _ptr(out), kv_heads_per_chunk,
                                        _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream),
                                        copy(stream2), copy(h2d_stream), copy(d2h_stream)))
+
+
+def qattn_tc_probe(kind, iters, n_ctas, cycles, dev_err, stream=None):
+    """Tensor-core peak probe (kind 0: INT8, 1: FP8 E4M3); see include/qattn_probe.h."""
+    _check(load().qattn_tc_probe(int(kind), int(iters), int(n_ctas), _ptr(cycles), _ptr(dev_err),
+                                 _stream(stream)))
 
 
 def qattn_check(dev_err, stream=None):

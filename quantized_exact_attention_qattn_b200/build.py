@@ -40,7 +40,7 @@ def needs_build() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-    deps.append(os.path.join(os.path.dirname(PKG), "include", "qattn.h"))
+    deps += glob.glob(os.path.join(os.path.dirname(PKG), "include", "*.h"))
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 

@@ -29,7 +29,44 @@ struct FwdParams {
   int B, Nq, Nkv, Hq, Hkv, G, nK, nQ, n_groups;
   float c;
   int stall_tile;   // test hook: K/V tile whose copy is never issued (-1: none)
+  int kcap;         // K rows per (batch, head) plane of k8 (>= Nkv)
+  int ks_stride;    // K scales per (batch, head) in k_scale
+  // score copy-out (qattn_scores only): n_dump requested (b, h, q_tile, k_tile)
+  // quads and one [128][64] INT32 slot per quad
+  const int4* dump_tiles;
+  int32_t* dump_out;
+  int n_dump;
 };
+
+// Score copy-out of the debug build of the mainloop (qattn_scores).  The thread
+// owning query row `row` holds NCOL consecutive scores of key tile t, starting at
+// column col0, as the softmax reads them: x[j] - bias is the exact INT32 score
+// (bias = 1.5 * 2^23 where S accumulated onto that preload, 0 where it was
+// converted).  Every slot whose request names (b, h, qt, t) receives them; the
+// warp's lanes scan the request list 32 entries at a time.
+template <int NCOL>
+__device__ __forceinline__ void dump_scores(const FwdParams& p, int b, int h, int qt, int t,
+                                            int row, int col0, const float (&x)[NCOL],
+                                            float bias) {
+  const int lane = threadIdx.x & 31;
+  for (int base = 0; base < p.n_dump; base += 32) {
+    bool hit = false;
+    if (base + lane < p.n_dump) {
+      const int4 r = p.dump_tiles[base + lane];
+      hit = r.x == b && r.y == h && r.z == qt && r.w == t;
+    }
+    uint32_t m = __ballot_sync(0xffffffffu, hit);
+    while (m) {
+      const int slot = base + __ffs(m) - 1;
+      m &= m - 1;
+      int4* dst = reinterpret_cast<int4*>(p.dump_out + (static_cast<int64_t>(slot) * BM + row) * 64 + col0);
+#pragma unroll
+      for (int j = 0; j < NCOL; j += 4)
+        dst[j / 4] = make_int4(__float2int_rn(__fsub_rn(x[j], bias)), __float2int_rn(__fsub_rn(x[j + 1], bias)),
+                               __float2int_rn(__fsub_rn(x[j + 2], bias)), __float2int_rn(__fsub_rn(x[j + 3], bias)));
+    }
+  }
+}
 
 // ---------------------------------------------------------------- exp2
 // Columns j with (j % 8) < kPolyPer8 evaluate 2^t with an FMA-pipe polynomial,
@@ -152,6 +189,26 @@ __device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
   }
 }
 
+// O <- O * o for the 64 O columns a thread owns in the two-threads-per-row layout
+// (16x32bx2 accesses: threads 0-15 columns 0-63 of their lanes, threads 16-31
+// columns 64-127), 32 columns at a time.
+__device__ __forceinline__ void rescale_halves(uint32_t tO, float o) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < 64; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld16x2_x32<64>(tO + c0, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                             make_float2(o, o));
+      r[j] = __float_as_uint(v.x);
+      r[j + 1] = __float_as_uint(v.y);
+    }
+    tmem_st16x2_x32<64>(tO + c0, r);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -170,6 +227,22 @@ inline EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(ptr);
   });
   return fn;
+}
+
+// 3-D uint8 tensor map with explicit pitches (bytes): extents {inner, rows, planes},
+// row_pitch and plane_pitch multiples of 16; reads past an extent return zeros.
+inline bool make_map_pitched(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                             uint64_t planes, uint64_t row_pitch, uint64_t plane_pitch,
+                             uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, rows, planes};
+  const cuuint64_t strides[2] = {row_pitch, plane_pitch};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 3-D uint8 tensor map: dims {inner, rows, planes}, row pitch = inner bytes.

@@ -2,10 +2,10 @@
 //
 // Numerics: "Exact Numerical Contract", sections "INT8 QK And Score Domain",
 // "Online Softmax", "V And PV", "Finalization And Tails".  Per query row and
-// per 64-key tile t (ascending):
-//   s = ((float)S * (q_scale * k_scale)) * c        S = Q8 K8^T (exact INT32)
+// per 64-key tile t (ascending), S = Q8 K8^T exact in INT32:
+//   A = (q_scale * k_scale) * c;  s = S * A          (FP32, c = log2(e) / sqrt(D))
 //   mn = max(m, max(s) - 8.807);  old = ex2(m - mn);  d *= old;  O *= old
-//   p = ex2(s - mn);  d += p;  P8 = e4m3(p);  O += P8 V8;  m = mn
+//   p = ex2(fma(S, A, -mn));  d += p;  P8 = e4m3(p);  O += P8 V8;  m = mn
 //   out = bf16(O * rcp(d) * v_scale)
 //
 // Blackwell mapping (one CTA = NQT query tiles of 128 rows of one (b, h)):
@@ -56,7 +56,14 @@ using namespace attn;
 
 constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
 
-template <int D, int NQT>
+#ifndef QATTN_D128_HALVES
+#define QATTN_D128_HALVES 0
+#endif
+
+// PV 0: FP8 E4M3 P and V (kind::f8f6f4), two P buffers of 16 columns per query
+// tile; PV 1: FP16 P and V (kind::f16), one P buffer of 32 columns (the same
+// tensor-memory columns) and V tiles of 64 keys x 2 bytes per dim row.
+template <int D, int NQT, int PV = 0>
 struct Cfg {
   static constexpr int STAGES = (D == 256) ? 3 : 4;
   static constexpr int KCH = (D >= 128) ? 128 : 64;        // K-major swizzle row width (bytes)
@@ -64,7 +71,8 @@ struct Cfg {
   static constexpr uint32_t SW_QK = (KCH == 128) ? 2u : 4u; // 128B or 64B swizzle
   static constexpr int Q_BYTES = BM * D;
   static constexpr int K_BYTES = BN * D;
-  static constexpr int V_BYTES = D * BN;
+  static constexpr int VB = PV ? 2 : 1;                     // bytes per V element
+  static constexpr int V_BYTES = D * BN * VB;
   // Q in tensor memory (A operand of QK read from TMEM, so each QK MMA reads only
   // its K tile from shared memory) wherever the columns allow: D = 128 with two
   // query tiles, D = 256 with one; D = 64 with three keeps Q in shared memory.
@@ -76,8 +84,11 @@ struct Cfg {
   // D = 256, where the longer P.V gives the softmax more time per tile and more
   // warps hide more of its latency) two per query tile, one per half of the keys.
   static constexpr bool SPLIT = (D == 256);
-  static constexpr int SM_WARPS = (SPLIT ? 8 : 4) * NQT;            // softmax warps
-  static constexpr int ARRIVALS = SPLIT ? 8 : 4;                    // softmax warps per query tile
+  // D = 128: two threads per query row inside one warp (16x32bx2 tensor-memory
+  // accesses), eight softmax warps per query tile, four per sub-partition in all
+  static constexpr bool HALVES = (D == 128) && (QATTN_D128_HALVES != 0);
+  static constexpr int SM_WARPS = ((SPLIT || HALVES) ? 8 : 4) * NQT;  // softmax warps
+  static constexpr int ARRIVALS = (SPLIT || HALVES) ? 8 : 4;          // softmax warps per query tile
   static constexpr int KS_PER_WARP = SPLIT ? 32 : 64;               // staged per-token K scales
   static constexpr int SMEM_KS = SMEM_V + STAGES * V_BYTES;         // float [softmax warps][KS_PER_WARP]
   static constexpr int SMEM_DEN = SMEM_KS + SM_WARPS * KS_PER_WARP * 4;  // float [NQT][2][128]
@@ -98,7 +109,8 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(Q_COL + (Q_TMEM ? NQT * (D / 4) : 0) <= TMEM_COLS, "tensor memory budget");
   static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
-  static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
+  // e4m3 x e4m3 -> f32 (kind::f8f6f4) or f16 x f16 -> f32 (kind::f16): format code 0 both
+  static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);
 };
 
 // Bytes b0 .. b0+127 of query row n (head bh) into 32 tensor-memory columns at taddr
@@ -124,11 +136,14 @@ __device__ __forceinline__ void store_q_row(const FwdParams& p, int bh, int n, i
   tmem_st32(taddr, r);
 }
 
-template <int D, int NQT, int KMODE>
-__global__ void __launch_bounds__(Cfg<D, NQT>::THREADS, 1)
+// DUMP: the debug build behind qattn_scores; it also copies the requested score
+// tiles out as the softmax warps recover them (dump_scores), and is otherwise the
+// same kernel.
+template <int D, int NQT, int KMODE, bool DUMP, int PV>
+__global__ void __launch_bounds__(Cfg<D, NQT, PV>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = Cfg<D, NQT>;
+  using C = Cfg<D, NQT, PV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -226,7 +241,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int ch = 0; ch < C::NCH; ++ch)
           tma_load_3d(smem + C::SMEM_K + s * C::K_BYTES + ch * (BN * C::KCH), &tmK, kv_full + s,
                       ch * C::KCH, t * BN, bhkv);
-        tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN, 0, bhkv);
+        tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN * C::VB, 0, bhkv);
         issued = t + 1;
       }
       int dummy = 0;      // drain: every issued copy must land before the CTA may exit
@@ -285,11 +300,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ok = mbar_wait(p_full + 2 * i + (t & 1), (t >> 1) & 1, abort, p.dev_err, kErrTimeoutP);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a_tm = tmem + C::P_COL + (i * 2 + (t & 1)) * (BN / 4);
+        if constexpr (PV == 0) {   // P_i(t) in buffer t & 1; V rows of 64 keys, 64-byte swizzle
+          const uint32_t a_tm = tmem + C::P_COL + (i * 2 + (t & 1)) * (BN / 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk) {
-          const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
-          mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 32; ++kk) {
+            const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 64, 4u);
+            mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {                   // one FP16 P buffer; V rows of 128 bytes, 128-byte swizzle
+          const uint32_t a_tm = tmem + C::P_COL + i * (BN / 2);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {   // K = 16 FP16 (32 bytes, 8 columns) per MMA
+            const uint64_t bd = smem_desc(sV + s * C::V_BYTES + kk * 32, 8 * 128, 2u);
+            mma_f16_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         tc_commit(pv_done + 2 * i + (t & 1));
         tc_commit(kv_empty + s);   // stage s is free once every issuer's reads finished
@@ -319,20 +343,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int qt = qt0 + i;
         const uint32_t tS = tmem + lane_off + C::S_COL + i * BN;
         const uint32_t tS_own = tS + hf * 32;
-        const uint32_t tP = tmem + lane_off + C::P_COL + (i * 2) * (BN / 4) + hf * (BN / 8);
+        // this half's 32 keys: 8 columns of P buffer (t & 1) (FP8) or 16 of the FP16 buffer
+        const uint32_t tP = tmem + lane_off + C::P_COL + i * (BN / 2) + hf * (PV ? BN / 4 : BN / 8);
         const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
         const int last_valid = p.Nkv - (nK - 1) * BN;
-        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
-        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
+        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const int n_groups32 = (p.Nkv + 31) / 32;        // scales per 32-row group (mode 2)
         float m = kMInit;
         float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
-        // per-token scales: lane l holds token 32 hf + l of a tile (0 past the end)
+        // per-key scales: lane l holds the scale of token 32 hf + l of a tile (0 past
+        // the end): its own (mode 1) or its 32-row group's (mode 2)
         auto load_kone = [&](int tt) {
-          const int j = tt * BN + hf * 32 + lane;
-          return j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f;
+          if constexpr (KMODE == 2) {
+            const int g = 2 * tt + hf;
+            return g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
+          } else {
+            const int j = tt * BN + hf * 32 + lane;
+            return j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f;
+          }
         };
         float kone_next = 0.0f;
-        if constexpr (KMODE == 1) kone_next = load_kone(0);
+        if constexpr (KMODE != 0) kone_next = load_kone(0);
         if constexpr (C::Q_TMEM) {   // this warp's rows, its half of the D bytes
           store_q_row(p, bh, qt * BM + row, D, hf * 128, tmem + lane_off + C::Q_COL + i * (D / 4) + hf * 32);
           tmem_wait_st();
@@ -346,7 +378,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const float ks_cur = ks_next;
           if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
           const float kone = kone_next;
-          if constexpr (KMODE == 1) {
+          if constexpr (KMODE != 0) {
             if (t + 1 < nK) kone_next = load_kone(t + 1);
           }
           ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, t & 1, abort, p.dev_err, kErrTimeoutS));
@@ -361,6 +393,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // INT32 scores to FP32: exact, |S| <= D * 127^2 < 2^24
 #pragma unroll
           for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
+          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, hf * 32, x, 0.0f);
           const bool last = (t == nK - 1);
           const int nv = last ? last_valid : BN;          // valid keys in this tile
           const int own0 = hf * 32;                       // first key of this half
@@ -456,9 +489,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           acc[2] = fadd2(acc[2], acc[3]);
           acc[0] = fadd2(acc[0], acc[2]);
           den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
-          uint32_t pk[8];
+          uint32_t pk[PV ? 16 : 8];
+          if constexpr (PV == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+            for (int j = 0; j < 32; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) pk[j / 2] = cvt_f16x2(x[j], x[j + 1]);
+          }
           if (t >= 1) {
             // PV_i(t-1) was issued when both halves finished tile t-1 and has long
             // completed.  Its completion frees P buffer (t & 1), last read by
@@ -470,7 +508,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_fence_after();
             if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D / 2>(tO, old);
           }
-          tmem_st8(tP + (t & 1) * (BN / 4), pk);
+          if constexpr (PV == 0)
+            tmem_st8(tP + (t & 1) * (BN / 4), pk);
+          else
+            tmem_st16(tP, pk);                            // PV_i(t-1) has read P_i(t-1)
           tmem_wait_st();                                 // P and any O rescale have landed
           tc_fence_before();
           __syncwarp();
@@ -488,7 +529,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           const float inv = rcp_approx(__fadd_rn(den_s[(i * 2) * BM + row], den_s[(i * 2 + 1) * BM + row]));
           const int n = qt * BM + row;
-          const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D + hf * (D / 2);
+          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + hf * (D / 2);
           uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + hf * (D / 2);
 #pragma unroll 1
           for (int c0 = 0; c0 < D / 2; c0 += 32) {
@@ -499,9 +540,250 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               uint32_t w[16];
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
-                const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                             make_float2(inv, inv)),
-                                       make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                 make_float2(inv, inv));
+                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+              }
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+              d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+              d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            }
+          }
+        }
+      }
+    } else if constexpr (C::HALVES) {
+      // ================================================================ softmax, D = 128
+      // Eight warps per query tile, two threads per row of the same warp.  Warp
+      // slot s = 0..7 of tile i covers lanes 32 (s % 4) + 16 (s / 4) .. +15 (its
+      // sub-partition's quadrant); of lane r's two threads, the first (thread r)
+      // owns keys 0-31 of each tile and O columns 0-63, the second (thread r + 16)
+      // keys 32-63 and O columns 64-127 (16x32bx2 accesses).  The row's tile
+      // maximum is one shuffle between the two; each keeps its own partial
+      // denominator, added at the end.
+      const int slot = warp - C::SOFTMAX_WARP0;
+      const int i = slot >> 3;
+      const int q4 = warp & 3;
+      const int hb = (slot >> 2) & 1;
+      const int kh = lane >> 4;
+      const int row = q4 * 32 + hb * 16 + (lane & 15);
+      if (i < nvalid) {
+        const int qt = qt0 + i;
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32 + hb * 16) << 16;
+        const uint32_t tS = tmem + lane_off + C::S_COL + i * BN;
+        const uint32_t tP = tmem + lane_off + C::P_COL + (i * 2) * (BN / 4);
+        const uint32_t tO = tmem + lane_off + C::O_COL + i * D;
+        const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
+        const int last_valid = p.Nkv - (nK - 1) * BN;
+        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const int n_groups32 = (p.Nkv + 31) / 32;        // scales per 32-row group (mode 2)
+        float m = kMInit;
+        float den = (kh == 0) ? 1.0f : 0.0f;   // the two halves' partial sums add up to d
+        float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
+        // per-key scales: lane l holds those of tokens 2l, 2l+1 of a tile (0 past the
+        // end): their own (mode 1) or their 32-row group's (mode 2)
+        auto load_kpair = [&](int tt) {
+          if constexpr (KMODE == 2) {
+            const int g = 2 * tt + (lane >> 4);
+            const float v = g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
+            return make_float2(v, v);
+          } else {
+            const int j = tt * BN + 2 * lane;
+            return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
+                               j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+          }
+        };
+        float2 kpair_next = make_float2(0.0f, 0.0f);
+        if constexpr (KMODE != 0) kpair_next = load_kpair(0);
+        {   // this thread's 64 bytes of its Q row into tensor memory (16 columns)
+          const int n = qt * BM + row;
+          uint32_t r[16];
+          if (n < p.Nq) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                p.q8 + (static_cast<int64_t>(bh) * p.Nq + n) * D + kh * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = __ldg(src + c);
+              r[4 * c] = v.x;
+              r[4 * c + 1] = v.y;
+              r[4 * c + 2] = v.z;
+              r[4 * c + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) r[c] = 0u;
+          }
+          tmem_st16x2_x16<16>(tmem + lane_off + C::Q_COL + i * (D / 4), r);
+        }
+        // S accumulates onto the bits of kMagic (1.5 * 2^23), read back as FP32 it is
+        // exactly kMagic + S (|S| < 2^22)
+        tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);
+        tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(q_ready + i);
+          mbar_arrive(s_free + i);                  // s_free phase t: QK_i(t) may accumulate
+        }
+        bool ok = true;
+        for (int t = 0; ok && t < nK; ++t) {
+          const float ks_cur = ks_next;
+          if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
+          const float2 kpair = kpair_next;
+          if constexpr (KMODE != 0) {
+            if (t + 1 < nK) kpair_next = load_kpair(t + 1);
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, t & 1, abort, p.dev_err, kErrTimeoutS));
+          if (!ok) break;
+          tc_fence_after();
+          float x[32];                                    // keys 32 kh .. 32 kh + 31
+          tmem_ld16x2_x32<32>(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+          tmem_wait_ld();
+          tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);     // reset S for QK_i(t+1)
+          tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + i);
+          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kMagic);
+          const bool last = (t == nK - 1);
+          const int k0 = kh * 32;                         // first key of this half
+          float mn;
+          float2 a2, nb2;
+          if constexpr (KMODE == 0) {
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (k0 + j >= last_valid) x[j] = -INFINITY;   // masked key: p = 0
+            }
+            float mq[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              mq[q] = fmaxf(x[16 * q], x[16 * q + 15]);
+#pragma unroll
+              for (int j = 1; j < 15; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
+            }
+            float xmax = fmaxf(mq[0], mq[1]);
+            xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 16));   // the row's other half
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
+            }
+            const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
+            a2 = make_float2(a, a);
+            nb2 = make_float2(-mn, -mn);
+          } else {
+            // per-token K scales: the warp stages the tile's 64 scales (two per lane);
+            // each half reads its own 32
+            const int nv = last ? last_valid : BN;
+            float* kss = ks_stage + slot * BN;
+            kss[2 * lane] = kpair.x;
+            kss[2 * lane + 1] = kpair.y;
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
+            }
+            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
+            float smx = -INFINITY;
+            if (!last) {
+              smx = kt_tile_max<32>(x, kss + k0, qs2, c2);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (k0 + j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[k0 + j]), p.c)));
+            }
+            smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, 16));
+            mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
+            nb2 = make_float2(-mn, -mn);
+          }
+          const float old = ex2_approx(__fsub_rn(m, mn));
+          if constexpr (KMODE == 0) {
+            exp_block<0, 32>(x, a2, nb2);
+          } else {
+            exp_block_kt<0, 32>(x, ks_stage + slot * BN + k0, make_float2(qs, qs),
+                                make_float2(p.c, p.c), nb2);
+            __syncwarp();                                 // kss is rewritten next tile
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (k0 + j >= last_valid) x[j] = 0.0f;    // masked key: p = 0
+            }
+          }
+          // partial denominator: unquantized probabilities, four independent pair sums
+          float2 acc[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
+#pragma unroll
+          for (int j = 8; j < 32; j += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
+          }
+          acc[0] = fadd2(acc[0], acc[1]);
+          acc[2] = fadd2(acc[2], acc[3]);
+          acc[0] = fadd2(acc[0], acc[2]);
+          den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
+          uint32_t pk[PV ? 16 : 8];
+          if constexpr (PV == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) pk[j / 2] = cvt_f16x2(x[j], x[j + 1]);
+          }
+          if (t >= 1) {
+            // PV_i(t-1) frees P buffer (t & 1), last read by PV_i(t-2), and must land
+            // before this thread rescales its half of the row's O by old
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
+                                                   abort, p.dev_err, kErrTimeoutO));
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_halves(tO, old);
+          }
+          if constexpr (PV == 0)
+            tmem_st16x2_x8<8>(tP + (t & 1) * (BN / 4), pk);   // keys 32 kh .. : columns 8 kh ..
+          else
+            tmem_st16x2_x16<16>(tP, pk);                     // keys 32 kh .. : columns 16 kh ..
+          tmem_wait_st();                                 // P and any O rescale have landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + 2 * i + (t & 1));
+          m = mn;
+        }
+        // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization")
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
+                                                 abort, p.dev_err, kErrTimeoutO));
+        den = __fadd_rn(den, __shfl_xor_sync(0xffffffffu, den, 16));   // d = d_0 + d_1
+        if (ok) {
+          tc_fence_after();
+          const float inv = rcp_approx(den);
+          const int n = qt * BM + row;
+          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + kh * 64;
+          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + kh * 64;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld16x2_x32<64>(tO + c0, o);
+            tmem_wait_ld();
+            if (n < p.Nq) {
+              uint32_t w[16];
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                 make_float2(inv, inv));
+                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
                 w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
                            (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
               }
@@ -527,18 +809,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t tO = tmem + lane_off + C::O_COL + wg * D;
         const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
         const int last_valid = p.Nkv - (nK - 1) * BN;
-        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * nK;
-        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.Nkv;
+        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
+        const int n_groups32 = (p.Nkv + 31) / 32;        // scales per 32-row group (mode 2)
         float m = kMInit, den = 1.0f;
         float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
-        // per-token scales: lane l holds tokens 2l, 2l+1 of a tile (0 past the end)
+        // per-key scales: lane l holds those of tokens 2l, 2l+1 of a tile (0 past the
+        // end): their own (mode 1) or their 32-row group's (mode 2)
         auto load_kpair = [&](int tt) {
-          const int j = tt * BN + 2 * lane;
-          return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
-                             j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+          if constexpr (KMODE == 2) {
+            const int g = 2 * tt + (lane >> 4);
+            const float v = g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
+            return make_float2(v, v);
+          } else {
+            const int j = tt * BN + 2 * lane;
+            return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
+                               j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+          }
         };
         float2 kpair_next = make_float2(0.0f, 0.0f);
-        if constexpr (KMODE == 1) kpair_next = load_kpair(0);
+        if constexpr (KMODE != 0) kpair_next = load_kpair(0);
         if constexpr (C::Q_TMEM) {   // this warp's rows of Q_i (D = 128: 32 columns)
           static_assert(!C::Q_TMEM || D == 128, "one 32-column store per row");
           store_q_row(p, bh, qt * BM + row, D, 0, tmem + lane_off + C::Q_COL + wg * (D / 4));
@@ -563,7 +853,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float ks_cur = ks_next;
           if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
           const float2 kpair = kpair_next;
-          if constexpr (KMODE == 1) {
+          if constexpr (KMODE != 0) {
             if (t + 1 < nK) kpair_next = load_kpair(t + 1);
           }
           ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
@@ -580,6 +870,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + wg);
+          if constexpr (DUMP) dump_scores<64>(p, b, h, qt, t, row, 0, x, kMagic);
           const bool last = (t == nK - 1);
           float mn;
           float2 a2, nb2;
@@ -664,9 +955,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           acc[2] = fadd2(acc[2], acc[3]);
           acc[0] = fadd2(acc[0], acc[2]);
           den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
-          uint32_t pk[16];
+          uint32_t pk[PV ? 32 : 16];
+          if constexpr (PV == 0) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+            for (int j = 0; j < 64; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) pk[j / 2] = cvt_f16x2(x[j], x[j + 1]);
+          }
           if (t >= 1) {
             // PV_i(t-1) was issued when this warpgroup finished tile t-1 and has long
             // completed.  Its completion frees P buffer (t & 1), last read by
@@ -678,7 +974,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_fence_after();
             if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D>(tO, old);
           }
-          tmem_st16(tP + (t & 1) * (BN / 4), pk);
+          if constexpr (PV == 0)
+            tmem_st16(tP + (t & 1) * (BN / 4), pk);
+          else
+            tmem_st32(tP, pk);
           tmem_wait_st();                                 // P and any O rescale have landed
           tc_fence_before();
           __syncwarp();
@@ -693,7 +992,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           const float inv = rcp_approx(den);
           const int n = qt * BM + row;
-          const float* vs = p.v_scale + static_cast<int64_t>(bhkv) * D;
+          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D;
           uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D;
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
@@ -704,9 +1003,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               uint32_t w[16];
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
-                const float2 v = fmul2(fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                             make_float2(inv, inv)),
-                                       make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
+                                 make_float2(inv, inv));
+                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
                 w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
                            (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
               }
@@ -730,189 +1029,95 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
-// ------------------------------------------------------------------ scores (debug)
-// One CTA per requested (b, h, q_tile, k_tile): TMA both tiles, the same
-// kind::i8 MMA sequence as the mainloop, tcgen05.ld of the INT32 tile.
-template <int D>
-__global__ void __launch_bounds__(128, 1)
-scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const int32_t* tiles, int32_t* s_out, int Hq, int Hkv, int* dev_err) {
-  using C = Cfg<D, 1>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::Q_BYTES;
-  __shared__ uint64_t bar_ld, bar_mma;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_flag;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t* tl = tiles + 4 * blockIdx.x;
-  const int b = tl[0], h = tl[1], qt = tl[2], kt = tl[3];
-  const int hkv = h / (Hq / Hkv);
-  if (threadIdx.x == 0) {
-    abort_flag = 0;
-    mbar_init(&bar_ld, 1);
-    mbar_init(&bar_mma, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, 64);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_sh;
-  volatile int* abort = &abort_flag;
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&bar_ld, static_cast<uint32_t>(C::Q_BYTES + C::K_BYTES));
-    for (int ch = 0; ch < C::NCH; ++ch) {
-      tma_load_3d(sQ + ch * (BM * C::KCH), &tmQ, &bar_ld, ch * C::KCH, qt * BM, b * Hq + h);
-      tma_load_3d(sK + ch * (BN * C::KCH), &tmK, &bar_ld, ch * C::KCH, kt * BN, b * Hkv + hkv);
-    }
-  }
-  if (threadIdx.x == 32) {
-    int dummy = 0;
-    if (mbar_wait(&bar_ld, 0, abort, dev_err, kErrTimeoutQ)) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk) {
-        const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
-        const uint64_t ad = smem_desc(smem_u32(sQ) + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK);
-        const uint64_t bd = smem_desc(smem_u32(sK) + ch * (BN * C::KCH) + off, 8 * C::KCH, C::SW_QK);
-        mma_i8_ss(tmem, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-      }
-    }
-    tc_commit(&bar_mma);
-    (void)dummy;
-  }
-  __syncwarp();
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_mma, 0, abort, dev_err, kErrTimeoutS));
-  {
-    int dummy = 0;   // the TMA must have landed before exit, whatever happened
-    if (threadIdx.x == 0) mbar_wait(&bar_ld, 0, &dummy, dev_err, kErrTimeoutDrain);
-  }
-  if (ok) {
-    tc_fence_after();
-    uint32_t r[64];
-    const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-    tmem_wait_ld();
-    int4* dst = reinterpret_cast<int4*>(s_out + (static_cast<int64_t>(blockIdx.x) * BM + warp * 32 + lane) * BN);
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      dst[j] = make_int4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 64);
-  }
-}
-
 // ------------------------------------------------------------------ host side
-template <int D, int NQT, int KMODE>
-cudaError_t launch_fwd_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
-                         const float* q_scale, const int8_t* k8, const void* k_scale,
-                         const uint8_t* v8t, const float* v_scale, float c, uint16_t* out,
-                         int* dev_err, cudaStream_t st, const char** why) {
-  using Cf = Cfg<D, NQT>;
-  const int nQ = (Nq + BM - 1) / BM;
-  const int nK = (Nkv + BN - 1) / BN;
+template <int D, int NQT, int KMODE, bool DUMP, int PV>
+cudaError_t launch_fwd_t(const FwdLaunch& L, const ScoreDump& dump, cudaStream_t st,
+                         const char** why) {
+  using Cf = Cfg<D, NQT, PV>;
+  const int nQ = (L.Nq + BM - 1) / BM;
+  const int nK = (L.Nkv + BN - 1) / BN;
+  const uint64_t BH = static_cast<uint64_t>(L.B) * L.Hkv;
   const CUtensorMapSwizzle swqk =
       (Cf::KCH == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap mQ, mK, mV;
-  if (!make_map(&mQ, q8, D, Nq, static_cast<uint64_t>(B) * Hq, Cf::KCH, BM, swqk) ||
-      !make_map(&mK, k8, D, Nkv, static_cast<uint64_t>(B) * Hkv, Cf::KCH, BN, swqk) ||
-      !make_map(&mV, v8t, static_cast<uint64_t>(nK) * BN, D, static_cast<uint64_t>(B) * Hkv, BN, D,
-                CU_TENSOR_MAP_SWIZZLE_64B)) {
+  bool ok = make_map(&mQ, L.q8, D, L.Nq, static_cast<uint64_t>(L.B) * L.Hq, Cf::KCH, BM, swqk) &&
+            make_map_pitched(&mK, L.k8, D, L.Nkv, BH, D, static_cast<uint64_t>(D) * L.kcap, Cf::KCH,
+                             BN, swqk);
+  if (PV == 0)   // E4M3 [B,Hkv,D,64*nK]: rows past Nkv hold zeros
+    ok = ok && make_map(&mV, L.v, static_cast<uint64_t>(nK) * BN, D, BH, BN, D,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+  else           // FP16 [B,Hkv,D,kcap]: keys past Nkv read as zeros (outside the extent)
+    ok = ok && make_map_pitched(&mV, L.v, static_cast<uint64_t>(L.Nkv) * 2, D, BH,
+                                static_cast<uint64_t>(L.kcap) * 2,
+                                static_cast<uint64_t>(L.kcap) * 2 * D, BN * 2, D,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (pointer alignment or size)";
     return cudaErrorInvalidValue;
   }
   FwdParams p{};
-  p.q8 = q8; p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale; p.out = out; p.dev_err = dev_err;
-  p.B = B; p.Nq = Nq; p.Nkv = Nkv; p.Hq = Hq; p.Hkv = Hkv;
+  p.q8 = L.q8; p.q_scale = L.q_scale; p.k_scale = L.k_scale; p.v_scale = L.v_scale; p.out = L.out;
+  p.dev_err = L.dev_err;
+  p.B = L.B; p.Nq = L.Nq; p.Nkv = L.Nkv; p.Hq = L.Hq; p.Hkv = L.Hkv;
   p.G = 4 * nQ; p.nK = nK; p.nQ = nQ; p.n_groups = (nQ + NQT - 1) / NQT;
-  p.c = c;
+  p.c = L.c;
+  p.kcap = L.kcap;
+  p.ks_stride = KMODE == 0 ? (L.kcap + 63) / 64 : (KMODE == 1 ? L.kcap : (L.kcap + 31) / 32);
   p.stall_tile = stall_tile();
+  p.dump_tiles = reinterpret_cast<const int4*>(dump.tiles);
+  p.dump_out = dump.s_out;
+  p.n_dump = dump.n_tiles;
   // at least 116 KB so that one CTA (and one 512-column TMEM allocation) owns an SM
   const int smem = (Cf::SMEM_BYTES + 1024 > 116 * 1024) ? Cf::SMEM_BYTES + 1024 : 116 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT, KMODE>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NQT, KMODE, DUMP, PV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(B) * Hq * p.n_groups);
-  attn_fwd_kernel<D, NQT, KMODE><<<grid, Cf::THREADS, smem, st>>>(mQ, mK, mV, p);
+  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(L.B) * L.Hq * p.n_groups);
+  attn_fwd_kernel<D, NQT, KMODE, DUMP, PV><<<grid, Cf::THREADS, smem, st>>>(mQ, mK, mV, p);
   return cudaGetLastError();
+}
+
+template <int D, int NQT, int KMODE>
+cudaError_t launch_fwd_k(const FwdLaunch& L, const ScoreDump* dump, cudaStream_t st,
+                         const char** why) {
+  const ScoreDump none{nullptr, 0, nullptr};
+  if (L.pv == 1) {
+    if (dump != nullptr) {
+      *why = "the score copy-out build exists for the FP8 P.V kernel only";
+      return cudaErrorInvalidValue;
+    }
+    return launch_fwd_t<D, NQT, KMODE, false, 1>(L, none, st, why);
+  }
+  if (dump == nullptr) return launch_fwd_t<D, NQT, KMODE, false, 0>(L, none, st, why);
+  return launch_fwd_t<D, NQT, KMODE, true, 0>(L, *dump, st, why);
 }
 
 template <int D, int NQT>
-cudaError_t launch_fwd_d(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
-                         const float* q_scale, const int8_t* k8, const void* k_scale,
-                         int k_scale_mode, const uint8_t* v8t, const float* v_scale, float c,
-                         uint16_t* out, int* dev_err, cudaStream_t st, const char** why) {
-  if (k_scale_mode == 0)
-    return launch_fwd_t<D, NQT, 0>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, v8t, v_scale, c,
-                                   out, dev_err, st, why);
-  return launch_fwd_t<D, NQT, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, v8t, v_scale, c,
-                                 out, dev_err, st, why);
-}
-
-template <int D>
-cudaError_t launch_scores_t(int B, int Nq, int Nkv, int Hq, int Hkv, const int8_t* q8,
-                            const int8_t* k8, const int32_t* tiles, int n_tiles, int32_t* s_out,
-                            int* dev_err, cudaStream_t st, const char** why) {
-  using Cf = Cfg<D, 1>;
-  const CUtensorMapSwizzle swqk =
-      (Cf::KCH == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUtensorMap mQ, mK;
-  if (!make_map(&mQ, q8, D, Nq, static_cast<uint64_t>(B) * Hq, Cf::KCH, BM, swqk) ||
-      !make_map(&mK, k8, D, Nkv, static_cast<uint64_t>(B) * Hkv, Cf::KCH, BN, swqk)) {
-    *why = "cuTensorMapEncodeTiled failed (pointer alignment or size)";
-    return cudaErrorInvalidValue;
+cudaError_t launch_fwd_d(const FwdLaunch& L, const ScoreDump* dump, cudaStream_t st,
+                         const char** why) {
+  switch (L.k_scale_mode) {
+    case 0: return launch_fwd_k<D, NQT, 0>(L, dump, st, why);
+    case 1: return launch_fwd_k<D, NQT, 1>(L, dump, st, why);
+    case 2: return launch_fwd_k<D, NQT, 2>(L, dump, st, why);
+    default:
+      *why = "k_scale_mode must be 0, 1 or 2";
+      return cudaErrorInvalidValue;
   }
-  const int smem = Cf::Q_BYTES + Cf::K_BYTES + 1024;
-  cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  scores_kernel<D><<<n_tiles, 128, smem, st>>>(mQ, mK, tiles, s_out, Hq, Hkv, dev_err);
-  return cudaGetLastError();
 }
 
 }  // namespace
 
 void set_stall_tile(int tile) { g_stall_tile.store(tile); }
 
-cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
-                       const float* q_scale, const int8_t* k8, const void* k_scale,
-                       int k_scale_mode, const uint8_t* v8t, const float* v_scale,
-                       float score_c, uint16_t* out, int* dev_err, cudaStream_t st,
+cudaError_t launch_fwd(const FwdLaunch& L, const ScoreDump* dump, cudaStream_t st,
                        const char** why) {
-  switch (D) {
+  switch (L.D) {
     case 64:   // three query tiles: O 192 + S 192 + P 96 of the 512 TMEM columns
-      return launch_fwd_d<64, 3>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode, v8t,
-                                 v_scale, score_c, out, dev_err, st, why);
+      return launch_fwd_d<64, 3>(L, dump, st, why);
     case 128:
-      return launch_fwd_d<128, 2>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
-                                  v8t, v_scale, score_c, out, dev_err, st, why);
+      return launch_fwd_d<128, 2>(L, dump, st, why);
     case 256:
-      return launch_fwd_d<256, 1>(B, Nq, Nkv, Hq, Hkv, q8, q_scale, k8, k_scale, k_scale_mode,
-                                  v8t, v_scale, score_c, out, dev_err, st, why);
-    default:
-      *why = "head dimension must be 64, 128 or 256";
-      return cudaErrorInvalidValue;
-  }
-}
-
-cudaError_t launch_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
-                          const int8_t* k8, const int32_t* tiles, int n_tiles, int32_t* s_out,
-                          int* dev_err, cudaStream_t st, const char** why) {
-  switch (D) {
-    case 64: return launch_scores_t<64>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
-    case 128: return launch_scores_t<128>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
-    case 256: return launch_scores_t<256>(B, Nq, Nkv, Hq, Hkv, q8, k8, tiles, n_tiles, s_out, dev_err, st, why);
+      return launch_fwd_d<256, 1>(L, dump, st, why);
     default:
       *why = "head dimension must be 64, 128 or 256";
       return cudaErrorInvalidValue;

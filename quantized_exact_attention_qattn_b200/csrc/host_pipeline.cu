@@ -1,4 +1,4 @@
-// host_pipeline.cu — the whole path (prep -> quant -> fwd, or the Hadamard
+// host_pipeline.cu — the whole path (fused prep + quant -> fwd, or the Hadamard
 // quant -> fwd) for inputs and output in host memory.  Every (batch, KV head) is
 // an independent problem (per-head norms, means, scales and softmax), so the KV
 // heads are cut into chunks that stream through two device buffer sets: while one
@@ -35,7 +35,7 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Byte offsets of one buffer set, sized for `ck` KV heads (ck * G query heads).
 struct SetLayout {
-  size_t q_in, k_in, v_in, qp, kp, q8, q_scale, k8, k_scale, k_mean, v8t, v_scale, qws, out;
+  size_t q_in, k_in, v_in, q8, q_scale, k8, k_scale, k_mean, v8t, v_scale, qws, out;
   size_t qws_bytes, bytes;
 };
 
@@ -53,8 +53,6 @@ SetLayout set_layout(int B, int Nq, int Nkv, int G, int ck, int D) {
   L.q_in = take(rq * cq * D * 2);
   L.k_in = take(rk * ck * D * 2);
   L.v_in = take(rk * ck * D * 2);
-  L.qp = take(rq * cq * D * 2);
-  L.kp = take(rk * ck * D * 2);
   L.q8 = take(rq * cq * D);
   L.q_scale = take(static_cast<size_t>(B) * cq * 4 * nQ * 4);
   L.k8 = take(rk * ck * D);
@@ -63,7 +61,9 @@ SetLayout set_layout(int B, int Nq, int Nkv, int G, int ck, int D) {
   L.k_mean = take(static_cast<size_t>(B) * ck * D * 4);
   L.v8t = take(static_cast<size_t>(B) * ck * D * 64 * nK);
   L.v_scale = take(static_cast<size_t>(B) * ck * D * 4);
-  L.qws_bytes = qattn_quant_workspace_bytes(B, Nkv, ck, D);
+  // the fused quantizer's scratch (its RoPE tables sized for rotary_dim = D, the
+  // largest); the Hadamard quantizer needs less
+  L.qws_bytes = qattn_prep_quant_workspace_bytes(B, Nkv, ck, D, D);
   L.qws = take(L.qws_bytes);
   L.out = take(rq * cq * D * 2);
   L.bytes = o;
@@ -153,15 +153,15 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
   cudaStream_t compute[2] = {cs, stream2 ? static_cast<cudaStream_t>(stream2) : cs};
   cudaStream_t hs = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : cs;
   cudaStream_t ds = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : cs;
-  cudaEvent_t ev[7];   // start, h2d[2], comp[2], d2h[2]
-  for (int i = 0; i < 7; ++i) {
+  cudaEvent_t ev[8];   // start, h2d[2], comp[2], d2h[2], join
+  for (int i = 0; i < 8; ++i) {
     cudaError_t e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
       return hcuda(e, "cudaEventCreateWithFlags");
     }
   }
-  cudaEvent_t e_start = ev[0], *e_h2d = ev + 1, *e_comp = ev + 3, *e_d2h = ev + 5;
+  cudaEvent_t e_start = ev[0], *e_h2d = ev + 1, *e_comp = ev + 3, *e_d2h = ev + 5, e_join = ev[7];
   qattn_status st = QATTN_OK;
   auto cu = [&](cudaError_t e, const char* where) {
     if (e != cudaSuccess && st == QATTN_OK) st = hcuda(e, where);
@@ -218,15 +218,10 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
                                 reinterpret_cast<uint16_t*>(base + L.k_scale), v8t, v_scale,
                                 base + L.qws, L.qws_bytes, xs);
     } else {
-      const qattn_bnhd qpv{base + L.qp, {sq[0], sq[1], sq[2], sq[3]}};
-      const qattn_bnhd kpv{base + L.kp, {sk[0], sk[1], sk[2], sk[3]}};
-      st = qattn_prep(B, Nq, qc, kc, D, qv, kv, q_weight, k_weight, eps, rotary_dim, rope_theta, 0,
-                      reinterpret_cast<uint16_t*>(base + L.qp), reinterpret_cast<uint16_t*>(base + L.kp), xs);
-      if (st == QATTN_OK)
-        st = qattn_quant(B, Nq, Nkv, qc, kc, D, qpv, kpv, vv, q8, q_scale, k8,
-                         reinterpret_cast<float*>(base + L.k_scale),
-                         reinterpret_cast<float*>(base + L.k_mean), v8t, v_scale, base + L.qws,
-                         L.qws_bytes, xs);
+      st = qattn_prep_quant(B, Nq, qc, kc, D, qv, kv, vv, q_weight, k_weight, eps, rotary_dim,
+                            rope_theta, 0, q8, q_scale, k8, reinterpret_cast<float*>(base + L.k_scale),
+                            reinterpret_cast<float*>(base + L.k_mean), v8t, v_scale, base + L.qws,
+                            L.qws_bytes, xs);
     }
     if (st == QATTN_OK)
       st = qattn_fwd(B, Nq, Nkv, qc, kc, D, q8, q_scale, k8, base + L.k_scale, hadamard ? 1 : 0,
@@ -243,10 +238,16 @@ qattn_status qattn_attention_host(int B, int Nq, int Nkv, int Hq, int Hkv, int D
     }
     cu(cudaEventRecord(e_d2h[s], ds), "cudaEventRecord");
   }
-  // `stream` ends after the last copies of both sets: synchronizing it (or
-  // qattn_check on it) covers the whole call
-  for (int s = 0; s < std::min(n_chunks, 2); ++s) cudaStreamWaitEvent(cs, e_d2h[s], 0);
-  for (int i = 0; i < 7; ++i) cudaEventDestroy(ev[i]);   // released once their work completes
+  // `stream` ends after everything this call queued on the other streams, on
+  // success and after an error alike (a chunk may fail after its copies were
+  // queued): synchronizing it (or qattn_check on it) covers the whole call, so the
+  // caller may then reuse the workspace and the host buffers
+  const cudaStream_t others[3] = {hs, ds, compute[1]};
+  for (cudaStream_t o : others) {
+    if (o == cs) continue;
+    if (cudaEventRecord(e_join, o) == cudaSuccess) cudaStreamWaitEvent(cs, e_join, 0);
+  }
+  for (int i = 0; i < 8; ++i) cudaEventDestroy(ev[i]);   // released once their work completes
   return st;
 }
 

@@ -12,6 +12,7 @@
 // while the token's row loads are already in flight.
 #include <cuda_bf16.h>
 
+#include "prep_row.cuh"
 #include "qattn_device.cuh"
 #include "qattn_internal.h"
 
@@ -37,28 +38,7 @@ struct PrepArgs {
   int64_t pos_offset;
 };
 
-// FP64 -> BF16 with one rounding: round |x| to the BF16 quantum of its binade
-// (2^(e-7), e = floor(log2|x|), or 2^-133 below the normal range), ties to even.
-__device__ __forceinline__ float bf16_round_f64(double x) {
-  if (x == 0.0) return static_cast<float>(x);
-  const double a = fabs(x);
-  int e = ilogb(a);
-  if (e < -126) e = -126;
-  const double quantum = ldexp(1.0, e - 7);
-  const double r = rint(a / quantum) * quantum;  // exact scaling by a power of two
-  return static_cast<float>(copysign(r, x));     // <= 8 significant bits: exact
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-// Two FP32 values -> one BF16 pair (x in the low half), each rounded to nearest even.
-__device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-}
+using namespace prep;
 
 template <int D>
 __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
@@ -103,16 +83,11 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
   // The first loads go out before the FP64 RoPE tables of all the CTA's tokens
   // are computed (by all threads at once), so the table latency overlaps them.
   load_passes(n0, 0);
-  for (int i = threadIdx.x; i < half; i += blockDim.x)
-    s_freq[i] = pow(a.theta, -(2.0 * i) / static_cast<double>(a.rotary_dim));
+  for (int i = threadIdx.x; i < half; i += blockDim.x) s_freq[i] = rope_freq(a.theta, i, a.rotary_dim);
   __syncthreads();
   for (int idx = threadIdx.x; idx < nt * half; idx += blockDim.x) {
     const int k = idx / half, i = idx - k * half;
-    const double ang = static_cast<double>(a.pos_offset + n0 + k) * s_freq[i];
-    double sv, cv;
-    sincos(ang, &sv, &cv);
-    s_cos[k][i] = bf16_round_f64(cv);
-    s_sin[k][i] = bf16_round_f64(sv);
+    rope_coef(a.pos_offset + n0 + k, s_freq[i], &s_cos[k][i], &s_sin[k][i]);
   }
   __syncthreads();
 
@@ -129,66 +104,19 @@ __global__ void __launch_bounds__(256) prep_kernel(const PrepArgs a) {
         const bool isq = hh < a.Hq;
         const int h = isq ? hh : hh - a.Hq;
         const uint16_t* w = isq ? a.qw : a.kw;
-        float x[8];
-        x[0] = bf16_lo(raw[pidx].x); x[1] = bf16_hi(raw[pidx].x);
-        x[2] = bf16_lo(raw[pidx].y); x[3] = bf16_hi(raw[pidx].y);
-        x[4] = bf16_lo(raw[pidx].z); x[5] = bf16_hi(raw[pidx].z);
-        x[6] = bf16_lo(raw[pidx].w); x[7] = bf16_hi(raw[pidx].w);
-
-        // ---- RMSNorm (skipped when this tensor has no weight; uniform per warp
-        //      only when Hq and Hkv rows do not share a warp, so every lane takes
-        //      part in the shuffles regardless)
-        float ss = __fmul_rn(x[0], x[0]);
-#pragma unroll
-        for (int e = 1; e < 8; ++e) ss = __fadd_rn(ss, __fmul_rn(x[e], x[e]));
-#pragma unroll
-        for (int off = L / 2; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-        // Packed FP32 pairs and BF16 pairs from here on: every element still sees
-        // exactly the same roundings (RN products, RN sums, BF16 RN) as above.
         uint32_t yb[4];                                  // BF16 pairs, dims 8l + 2j, 8l + 2j + 1
-        if (w != nullptr) {
-          const float ms = __fmul_rn(ss, 1.0f / D);
-          const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, a.eps)));
-          const uint4 wr = *reinterpret_cast<const uint4*>(w + 8 * l);
-          const uint32_t wv[4] = {wr.x, wr.y, wr.z, wr.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t xr = bf16x2_rn(fmul2(make_float2(x[2 * j], x[2 * j + 1]), make_float2(r, r)));
-            yb[j] = bf16x2_rn(fmul2(unpack_bf16x2(xr), unpack_bf16x2(wv[j])));
-          }
-        } else {
-          const uint32_t xv[4] = {raw[pidx].x, raw[pidx].y, raw[pidx].z, raw[pidx].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) yb[j] = xv[j];
-        }
-
-        // ---- split-half RoPE: lane l < R/16 pairs with lane l + R/16.  Both halves
-        //      as y*cos + o*sv, sv = -sin (first half) or +sin (second half), which
-        //      is bit for bit y*cos - o*sin or y*cos + o*sin; other lanes pass through.
+        rmsnorm8<D>(raw[pidx], w, a.eps, l, yb);
         if (rot_lanes > 0) {
-          const int pl = (l < half_lanes) ? l + half_lanes : (l < rot_lanes ? l - half_lanes : l);
-          const int src_lane = sub * L + pl;
-          uint32_t ob[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) ob[j] = __shfl_sync(0xffffffffu, yb[j], src_lane);
+          float cv[8], sn[8];
           if (l < rot_lanes) {
-            const bool first = l < half_lanes;
-            const int i0 = first ? 8 * l : 8 * l - half;
-            const float4 c0 = *reinterpret_cast<const float4*>(&s_cos[k][i0]);
-            const float4 c1 = *reinterpret_cast<const float4*>(&s_cos[k][i0 + 4]);
-            const float4 n0 = *reinterpret_cast<const float4*>(&s_sin[k][i0]);
-            const float4 n1 = *reinterpret_cast<const float4*>(&s_sin[k][i0 + 4]);
-            const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            const float sn = first ? -1.0f : 1.0f;       // exact sign flip
-            const float sv[8] = {sn * n0.x, sn * n0.y, sn * n0.z, sn * n0.w,
-                                 sn * n1.x, sn * n1.y, sn * n1.z, sn * n1.w};
+            const int i0 = l < half_lanes ? 8 * l : 8 * l - half;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 yc = fmul2(unpack_bf16x2(yb[j]), make_float2(cv[2 * j], cv[2 * j + 1]));
-              const float2 os = fmul2(unpack_bf16x2(ob[j]), make_float2(sv[2 * j], sv[2 * j + 1]));
-              yb[j] = bf16x2_rn(fadd2(yc, os));
+            for (int e = 0; e < 8; ++e) {
+              cv[e] = s_cos[k][i0 + e];
+              sn[e] = s_sin[k][i0 + e];
             }
           }
+          rope8(yb, sub, l, L, half_lanes, rot_lanes, cv, sn);
         }
 
         if (valid) {

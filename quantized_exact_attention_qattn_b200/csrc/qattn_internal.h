@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/qattn.h"
+#include "../../include/qattn_probe.h"
 
 namespace qattn {
 
@@ -19,6 +20,8 @@ inline BNHD to_bnhd(const qattn_bnhd& v) {
 
 // qattn_api.cu: record the thread-local message returned by qattn_last_error()
 void set_last_error(const char* msg);
+// qattn_api.cu: QATTN_OK on a compute capability 10.0 device, else a named refusal
+qattn_status require_sm100();
 
 // prep.cu
 cudaError_t launch_prep(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD k,
@@ -40,7 +43,19 @@ cudaError_t launch_kv_stats(int B, int Nkv, int Hkv, int D, const BNHD* kp, BNHD
 cudaError_t launch_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD qp, BNHD kp,
                          BNHD v, const float* k_mean, const float* vfac, int8_t* q8,
                          float* q_scale, int8_t* k8, float* k_scale, uint8_t* v8t,
-                         cudaStream_t st);
+                         cudaStream_t st, int k_rows = 64);
+cudaError_t launch_hadamard_part(int B, int N, int H, int D, BNHD x, bool is_q, int8_t* x8,
+                                 void* scale, int kcap, int key0, cudaStream_t st);
+// FP16 V, dim-major [B, Hkv, D, cap]: source rows -> keys key0 .. key0 + n_write
+cudaError_t launch_quant_v16(int B, int n_src, int Hkv, int D, BNHD v, int cap, int key0,
+                             int n_write, uint16_t* v16t, cudaStream_t st);
+// fused path: workspace = quant workspace, then BF16 cos / sin tables [N][R/2]
+size_t prep_quant_table_bytes(int N, int rotary_dim);
+cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD k, BNHD v,
+                              const uint16_t* qw, const uint16_t* kw, float eps, int rotary_dim,
+                              double theta, int64_t pos_offset, int8_t* q8, float* q_scale,
+                              int8_t* k8, float* k_scale, float* k_mean, uint8_t* v8t,
+                              float* v_scale, void* ws, cudaStream_t st);
 cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD q,
                                   BNHD k, BNHD v, const float* vfac, int8_t* q8,
                                   float* q_scale, int8_t* k8, uint16_t* k_scale16,
@@ -51,13 +66,42 @@ cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
 void set_stall_tile(int tile);
 int stall_tile();
 
-cudaError_t launch_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
-                       const float* q_scale, const int8_t* k8, const void* k_scale,
-                       int k_scale_mode, const uint8_t* v8t, const float* v_scale,
-                       float score_c, uint16_t* out, int* dev_err, cudaStream_t st,
+// Score copy-out requested by qattn_scores: n_tiles (b, h, q_tile, k_tile) quads
+// (device, 16-byte aligned) and an INT32 [n_tiles][128][64] destination.
+struct ScoreDump {
+  const int32_t* tiles;
+  int n_tiles;
+  int32_t* s_out;
+};
+
+// One attention launch.  k8 rows and k_scale entries per (batch, KV head) are
+// spaced kcap (>= Nkv) apart: kcap = Nkv for a plain problem, the allocated length
+// for a cache of which the first Nkv keys are used.  pv 0: v = E4M3
+// [B,Hkv,D,64*ceil(Nkv/64)] with v_scale; pv 1: v = FP16 [B,Hkv,D,kcap], no scale.
+// k_scale_mode 0: FP32 per 64 rows, 1: FP16 per token, 2: FP32 per 32 rows.
+struct FwdLaunch {
+  int B, Nq, Nkv, Hq, Hkv, D;
+  const int8_t* q8;
+  const float* q_scale;
+  const int8_t* k8;
+  const void* k_scale;
+  int k_scale_mode;
+  const void* v;
+  const float* v_scale;
+  int pv;
+  int kcap;
+  float c;             // log2(e) * softmax scale
+  uint16_t* out;
+  int* dev_err;
+};
+
+// dump == nullptr: the production kernel; otherwise its debug build that also
+// copies the requested score tiles out.
+cudaError_t launch_fwd(const FwdLaunch& L, const ScoreDump* dump, cudaStream_t st,
                        const char** why);
-cudaError_t launch_scores(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
-                          const int8_t* k8, const int32_t* tiles, int n_tiles, int32_t* s_out,
-                          int* dev_err, cudaStream_t st, const char** why);
+
+// tc_probe.cu
+cudaError_t launch_tc_probe(int kind, int iters, int n_ctas, unsigned long long* cycles,
+                            int* dev_err, cudaStream_t st);
 
 }  // namespace qattn

@@ -14,6 +14,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "prep_row.cuh"
 #include "qattn_device.cuh"
 #include "qattn_internal.h"
 
@@ -168,14 +169,56 @@ struct QuantArgs {
   uint8_t* v8t;
   int B, Nq, Nkv, Hq, Hkv, G, nK;
   int nq_blocks, nk_blocks, nv_blocks;
+  int k_rows;              // rows per K scale: 64, or 32 (scales per 32-row group)
+  int nK_scale;            // K scales per (batch, head): ceil(Nkv / k_rows)
+  // kp holds RAW K rows to be prepared here (RMSNorm with kw, RoPE from the
+  // coefficient tables) before the mean is subtracted; the fused path
+  bool k_raw;
+  const uint16_t* kw;
+  float eps;
+  int rotary_dim;
+  const uint16_t* cos_t;   // BF16 [Nkv][rotary_dim/2]
+  const uint16_t* sin_t;
 };
+
+// RoPE coefficients of the lane's 8 pairs at token n from the BF16 tables
+// [N][R/2] (R a multiple of 16, so the lane's 8 entries are one 16-byte chunk).
+__device__ __forceinline__ void table_coefs(const uint16_t* cos_t, const uint16_t* sin_t, int n,
+                                            int half, int l, int half_lanes, float (&cv)[8],
+                                            float (&sn)[8]) {
+  const int i0 = l < half_lanes ? 8 * l : 8 * l - half;
+  unpack8(*reinterpret_cast<const uint4*>(cos_t + static_cast<int64_t>(n) * half + i0), cv);
+  unpack8(*reinterpret_cast<const uint4*>(sin_t + static_cast<int64_t>(n) * half + i0), sn);
+}
+
+// RMSNorm + RoPE of one raw row chunk in the row layout of prep_row.cuh (L = D/8
+// lanes per row); `n` must index a valid table row (callers clamp it).
+template <int D>
+__device__ __forceinline__ uint4 prep_chunk(const uint4 raw, const uint16_t* w, float eps,
+                                            int rotary_dim, const uint16_t* cos_t,
+                                            const uint16_t* sin_t, int n) {
+  constexpr int L = D / 8;
+  const int lane = threadIdx.x & 31, sub = lane / L, l = lane - sub * L;
+  uint32_t yb[4];
+  prep::rmsnorm8<D>(raw, w, eps, l, yb);
+  const int rot_lanes = rotary_dim / 8, half = rotary_dim / 2, half_lanes = half / 8;
+  if (rot_lanes > 0) {
+    float cv[8], sn[8];
+    if (l < rot_lanes) table_coefs(cos_t, sin_t, n, half, l, half_lanes, cv, sn);
+    prep::rope8(yb, sub, l, L, half_lanes, rot_lanes, cv, sn);
+  }
+  return make_uint4(yb[0], yb[1], yb[2], yb[3]);
+}
 
 // A group of ROWS rows x D dims of one (batch, head): amax over valid rows,
 // one scale, int8 rows written head-major [B, H, N, D].
+// With `pa` (the fused path) the rows are raw K and are first prepared here
+// (RMSNorm + RoPE, the same arithmetic as qattn_prep); chunk c of thread t is
+// row (t + 128c) / (D/8), which is the row layout of prep_row.cuh.
 template <int D, int ROWS>
 __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, int b, int h,
                                             int H, int N, int row0, int8_t* dst8, float* scale_out,
-                                            float* red) {
+                                            float* red, const QuantArgs* pa = nullptr) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int CH = ROWS * CPR / 128;       // chunks per thread
   // The raw BF16 chunks stay in registers (4 per chunk) and are unpacked twice,
@@ -188,6 +231,14 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
     const int n = row0 + r;
     raw[c] = (n < N) ? *reinterpret_cast<const uint4*>(row_ptr(src, b, n, h) + d0)
                      : make_uint4(0, 0, 0, 0);
+  }
+  if (pa != nullptr) {
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int n = row0 + (threadIdx.x + c * 128) / CPR;
+      raw[c] = prep_chunk<D>(raw[c], pa->kw, pa->eps, pa->rotary_dim, pa->cos_t, pa->sin_t,
+                             n < N ? n : 0);
+    }
   }
   auto values = [&](int c, float (&x)[8]) {
     const int id = threadIdx.x + c * 128;
@@ -245,11 +296,16 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
   }
   blk -= a.nq_blocks;
   if (blk < a.nk_blocks) {                               // ---- K blocks
-    const int j = blk % a.nK, bh = blk / a.nK;
+    const int j = blk % a.nK_scale, bh = blk / a.nK_scale;
     const int h = bh % a.Hkv, b = bh / a.Hkv;
-    quant_group<D, kKvRows>(a.kp, a.k_mean + static_cast<int64_t>(bh) * D, b, h, a.Hkv, a.Nkv,
-                            j * kKvRows, a.k8, a.k_scale + static_cast<int64_t>(bh) * a.nK + j,
-                            red);
+    const float* mean = a.k_mean + static_cast<int64_t>(bh) * D;
+    float* sc = a.k_scale + static_cast<int64_t>(bh) * a.nK_scale + j;
+    if (a.k_rows == kKvRows)
+      quant_group<D, kKvRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kKvRows, a.k8, sc, red,
+                              a.k_raw ? &a : nullptr);
+    else
+      quant_group<D, kQRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kQRows, a.k8, sc, red,
+                             a.k_raw ? &a : nullptr);
     return;
   }
   blk -= a.nk_blocks;
@@ -301,6 +357,212 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
       *reinterpret_cast<uint4*>(dst + d * npad + c * 16) =
           *reinterpret_cast<const uint4*>(tile + d * kKvRows + c * 16);
     }
+  }
+}
+
+// ---------------------------------------------------------------- fused prep + quant
+// RoPE coefficient tables for positions pos_offset + n, n < N: BF16 cos / sin of
+// pos * theta^(-2i/R) (FP64, rounded once), [N][R/2] each.
+__global__ void rope_table_kernel(int N, int rotary_dim, double theta, int64_t pos_offset,
+                                  uint16_t* cos_t, uint16_t* sin_t) {
+  const int half = rotary_dim / 2;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(N) * half) return;
+  const int n = static_cast<int>(idx / half), i = static_cast<int>(idx - static_cast<int64_t>(n) * half);
+  float c, sv;
+  prep::rope_coef(pos_offset + n, prep::rope_freq(theta, i, rotary_dim), &c, &sv);
+  cos_t[idx] = static_cast<uint16_t>(__float_as_uint(c) >> 16);    // exact: c is a BF16 value
+  sin_t[idx] = static_cast<uint16_t>(__float_as_uint(sv) >> 16);
+}
+
+struct PrepStatsArgs {
+  BNHD q, k, v;                 // raw BF16 inputs
+  const uint16_t* qw;
+  const uint16_t* kw;
+  float eps;
+  int rotary_dim;
+  const uint16_t* cos_t;
+  const uint16_t* sin_t;
+  int8_t* q8;
+  float* q_scale;
+  double* ksum;                 // [B, nK, Hkv*D]
+  float* vmax;                  // [B, nK, Hkv*D]
+  int B, N, Hq, Hkv, G, nK;
+};
+
+// First pass of the fused path, one CTA (256 threads) per (64-row block j, batch,
+// KV head): the block's rows of the KV head's Hq/Hkv query heads are prepared and
+// quantized at once (their two 32-row groups, "Q And K Quantization"); its K rows
+// are prepared and their FP64 column sums taken over the block in ascending row
+// order (the partials of the K mean, "Preparation" step 4); its V rows give the
+// block's column maxima of |v| ("V And PV").  Q leaves as INT8 with no BF16 copy;
+// K is prepared again from the raw rows by the quantizer's second pass.
+template <int D>
+__global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) {
+  constexpr int L = D / 8, HPW = 32 / L;       // lanes per row, rows per warp
+  constexpr int RPP = 8 * HPW;                 // rows per pass (8 warps)
+  constexpr int PASSES = kKvRows / RPP;
+  __shared__ float red[2][8];
+  __shared__ __align__(16) uint16_t sK[kKvRows * D];   // the block's prepared K rows
+  __shared__ unsigned vmx[D];                          // |v| column maxima (FP32 bits)
+  const int j = blockIdx.x;
+  const int bhk = blockIdx.y, b = bhk / a.Hkv, hk = bhk - b * a.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / L, l = lane - sub * L;
+  const int n0 = j * kKvRows;
+  const int nv = min(kKvRows, a.N - n0);              // valid rows of the block
+  const int Gh = a.Hq / a.Hkv;
+  if (threadIdx.x < D) vmx[threadIdx.x] = 0u;
+  auto row_of = [&](int p) { return p * RPP + warp * HPW + sub; };
+
+  uint4 kraw[PASSES], vraw[PASSES];
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int n = n0 + row_of(p);
+    kraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.k, b, n, hk) + 8 * l)
+                      : make_uint4(0, 0, 0, 0);
+    vraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.v, b, n, hk) + 8 * l)
+                      : make_uint4(0, 0, 0, 0);
+  }
+
+  // ---- Q: prepare, group maxima, INT8 codes
+  for (int gi = 0; gi < Gh; ++gi) {
+    const int h = hk * Gh + gi;
+    uint4 y[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const int n = n0 + row_of(p);
+      y[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.q, b, n, h) + 8 * l)
+                     : make_uint4(0, 0, 0, 0);
+    }
+    float gmax[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const int n = n0 + row_of(p);
+      y[p] = prep_chunk<D>(y[p], a.qw, a.eps, a.rotary_dim, a.cos_t, a.sin_t, n < a.N ? n : 0);
+      if (n < a.N) {                                // rows past the end take no part
+        float x[8];
+        unpack8(y[p], x);
+        const int g = (p * RPP) / kQRows;             // a pass lies inside one group
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gmax[g] = fmaxf(gmax[g], fabsf(x[e]));
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) gmax[g] = fmaxf(gmax[g], __shfl_xor_sync(0xffffffffu, gmax[g], off));
+      if (lane == 0) red[g][warp] = gmax[g];
+    }
+    __syncthreads();
+    float f[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      float m = red[g][0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[g][w]);
+      m = fmaxf(1e-7f, m);                          // a group with no row: 1e-7f
+      f[g] = __fdiv_rn(127.0f, m);
+      if (threadIdx.x == g)
+        a.q_scale[(static_cast<int64_t>(b) * a.Hq + h) * a.G + 2 * j + g] = __fdiv_rn(m, 127.0f);
+    }
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const int n = n0 + row_of(p);
+      if (n < a.N) {
+        const float fg = f[(p * RPP) / kQRows];
+        float x[8];
+        unpack8(y[p], x);
+        int8_t q[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[e] = q8_of(__fmul_rn(x[e], fg));
+        uint2 o;
+        o.x = pack4_s8(q[0], q[1], q[2], q[3]);
+        o.y = pack4_s8(q[4], q[5], q[6], q[7]);
+        *reinterpret_cast<uint2*>(a.q8 + ((static_cast<int64_t>(b) * a.Hq + h) * a.N + n) * D + 8 * l) = o;
+      }
+    }
+    __syncthreads();                                // red is reused
+  }
+  // groups of the last 128-row tile past the last 64-row block hold no row
+  if (j == a.nK - 1) {
+    const int extra = a.G - 2 * a.nK;
+    for (int id = threadIdx.x; id < extra * Gh; id += blockDim.x) {
+      const int h = hk * Gh + id / extra, g = 2 * a.nK + id % extra;
+      a.q_scale[(static_cast<int64_t>(b) * a.Hq + h) * a.G + g] = __fdiv_rn(1e-7f, 127.0f);
+    }
+  }
+
+  // ---- K: prepare into shared memory; V: column maxima
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int r = row_of(p), n = n0 + r;
+    const uint4 y = prep_chunk<D>(kraw[p], a.kw, a.eps, a.rotary_dim, a.cos_t, a.sin_t,
+                                  n < a.N ? n : 0);
+    *reinterpret_cast<uint4*>(sK + r * D + 8 * l) = y;
+  }
+  float vm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    if (n0 + row_of(p) < a.N) {
+      float x[8];
+      unpack8(vraw[p], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) vm[e] = fmaxf(vm[e], fabsf(x[e]));
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int off = L; off < 32; off <<= 1) vm[e] = fmaxf(vm[e], __shfl_xor_sync(0xffffffffu, vm[e], off));
+  }
+  __syncthreads();                                  // vmx zeroed, sK written
+  if (sub == 0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicMax(&vmx[8 * l + e], __float_as_uint(vm[e]));   // |v| >= 0
+  }
+  // FP64 column sums over the block's valid rows, ascending (one column per thread)
+  const int C = a.Hkv * D;
+  const size_t o = (static_cast<size_t>(b) * a.nK + j) * C + static_cast<size_t>(hk) * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double s = 0.0;
+    for (int r = 0; r < nv; ++r) s = __dadd_rn(s, static_cast<double>(__uint_as_float(static_cast<uint32_t>(sK[r * D + d]) << 16)));
+    a.ksum[o + d] = s;
+  }
+  __syncthreads();                                  // every atomicMax landed
+  for (int d = threadIdx.x; d < D; d += blockDim.x) a.vmax[o + d] = __uint_as_float(vmx[d]);
+}
+
+// ---------------------------------------------------------------- FP16 V
+// V for the FP16 P.V product: BF16 -> FP16 round to nearest even, no scale,
+// stored dim-major [B, Hkv, D, cap] (keys contiguous).  One CTA per 64-key tile
+// of one (batch, head): source rows 0 .. n_src-1 go to keys key0 .. of the
+// destination; keys key0 + [n_src, n_write) are written as 0 (n_write a multiple
+// of 8 and key0 + n_write <= cap, both checked by the caller), keys outside
+// [key0, key0 + n_write) are not touched.
+template <int D>
+__global__ void __launch_bounds__(128) quant_v16_kernel(BNHD v, int n_src, int Hkv, int cap,
+                                                        int key0, int n_write, uint16_t* v16t) {
+  __shared__ __align__(16) uint16_t tile[D * kKvRows];   // [d][key]
+  const int j = blockIdx.x, bh = blockIdx.y, b = bh / Hkv, h = bh - b * Hkv;
+  constexpr int CPR = D / 8;
+  for (int id = threadIdx.x; id < kKvRows * CPR; id += blockDim.x) {
+    const int r = id / CPR, d0 = (id - r * CPR) * 8, n = j * kKvRows + r;
+    const uint4 raw = n < n_src ? *reinterpret_cast<const uint4*>(row_ptr(v, b, n, h) + d0)
+                                : make_uint4(0, 0, 0, 0);
+    float x[8];
+    unpack8(raw, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[(d0 + e) * kKvRows + r] = __half_as_ushort(__float2half_rn(x[e]));
+  }
+  __syncthreads();
+  const int kmax = min(kKvRows, n_write - j * kKvRows);  // keys of this tile to write (multiple of 8)
+  uint16_t* dst = v16t + static_cast<int64_t>(bh) * D * cap + key0 + j * kKvRows;
+  for (int id = threadIdx.x; id < D * (kKvRows / 8); id += blockDim.x) {
+    const int d = id / (kKvRows / 8), c = id - d * (kKvRows / 8);
+    if (c * 8 < kmax)
+      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(d) * cap + c * 8) =
+          *reinterpret_cast<const uint4*>(tile + d * kKvRows + c * 8);
   }
 }
 
@@ -376,6 +638,7 @@ struct HadArgs {
   uint16_t* k_scale16;
   int B, Nq, Nkv, Hq, Hkv, G;
   int nq_blocks, nk_blocks;
+  int kcap, key0;      // K rows land at key0 + n of planes of kcap rows (a key cache)
 };
 
 // Q: one CTA (8 warps, 4 rows each) per 32-row group; K: one warp per token.
@@ -433,8 +696,9 @@ __global__ void __launch_bounds__(256) hadamard_quant_kernel(const HadArgs a) {
   for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   amax = fmaxf(1e-7f, amax);
   const float f = __fdiv_rn(127.0f, amax);
-  if (lane == 0) a.k_scale16[tok] = __half_as_ushort(__float2half_rn(__fdiv_rn(amax, 127.0f)));
-  store_q8_e<D>(a.k8 + tok * D, v, f);
+  const int64_t slot = static_cast<int64_t>(bh) * a.kcap + a.key0 + n;   // destination row
+  if (lane == 0) a.k_scale16[slot] = __half_as_ushort(__float2half_rn(__fdiv_rn(amax, 127.0f)));
+  store_q8_e<D>(a.k8 + slot * D, v, f);
 }
 
 }  // namespace
@@ -479,8 +743,10 @@ cudaError_t launch_kv_stats(int B, int Nkv, int Hkv, int D, const BNHD* kp, BNHD
 cudaError_t launch_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD qp, BNHD kp,
                          BNHD v, const float* k_mean, const float* vfac, int8_t* q8,
                          float* q_scale, int8_t* k8, float* k_scale, uint8_t* v8t,
-                         cudaStream_t st) {
+                         cudaStream_t st, int k_rows) {
   QuantArgs a{};
+  a.k_rows = k_rows;
+  a.nK_scale = (Nkv + k_rows - 1) / k_rows;
   a.qp = qp; a.kp = kp; a.v = v;
   a.k_mean = k_mean; a.vfac = vfac;
   a.q8 = q8; a.q_scale = q_scale; a.k8 = k8; a.k_scale = k_scale; a.v8t = v8t;
@@ -488,13 +754,110 @@ cudaError_t launch_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD qp
   a.G = 4 * ((Nq + 127) / 128);
   a.nK = (Nkv + kKvRows - 1) / kKvRows;
   a.nq_blocks = q8 ? B * Hq * a.G : 0;
-  a.nk_blocks = k8 ? B * Hkv * a.nK : 0;
-  a.nv_blocks = B * Hkv * a.nK;
+  a.nk_blocks = k8 ? B * Hkv * a.nK_scale : 0;
+  a.nv_blocks = v8t ? B * Hkv * a.nK : 0;
   const unsigned grid = static_cast<unsigned>(a.nq_blocks + a.nk_blocks + a.nv_blocks);
   switch (D) {
     case 64: quant_kernel<64><<<grid, 128, 0, st>>>(a); break;
     case 128: quant_kernel<128><<<grid, 128, 0, st>>>(a); break;
     case 256: quant_kernel<256><<<grid, 128, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+size_t prep_quant_table_bytes(int N, int rotary_dim) {
+  return ((static_cast<size_t>(N) * (rotary_dim / 2) * sizeof(uint16_t) + 255) & ~static_cast<size_t>(255)) * 2;
+}
+
+cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD k, BNHD v,
+                              const uint16_t* qw, const uint16_t* kw, float eps, int rotary_dim,
+                              double theta, int64_t pos_offset, int8_t* q8, float* q_scale,
+                              int8_t* k8, float* k_scale, float* k_mean, uint8_t* v8t,
+                              float* v_scale, void* ws, cudaStream_t st) {
+  const int nK = (N + kKvRows - 1) / kKvRows;
+  QuantWorkspace w = carve_workspace(ws, B, N, Hkv, D);
+  uint16_t* cos_t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + quant_workspace_bytes(B, N, Hkv, D));
+  uint16_t* sin_t = cos_t + prep_quant_table_bytes(N, rotary_dim) / 2 / sizeof(uint16_t);
+  cudaError_t e;
+  if (rotary_dim > 0) {
+    const int64_t cnt = static_cast<int64_t>(N) * (rotary_dim / 2);
+    rope_table_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, st>>>(
+        N, rotary_dim, theta, pos_offset, cos_t, sin_t);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  PrepStatsArgs pa{q, k, v, qw, kw, eps, rotary_dim, cos_t, sin_t, q8, q_scale, w.ksum, w.vmax,
+                   B, N, Hq, Hkv, 4 * ((N + 127) / 128), nK};
+  const dim3 grid(nK, B * Hkv);
+  switch (D) {
+    case 64: prep_stats_kernel<64><<<grid, 256, 0, st>>>(pa); break;
+    case 128: prep_stats_kernel<128><<<grid, 256, 0, st>>>(pa); break;
+    case 256: prep_stats_kernel<256><<<grid, 256, 0, st>>>(pa); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int C = Hkv * D;
+  const int64_t cols = static_cast<int64_t>(B) * C;
+  kv_finalize_kernel<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+      B, N, nK, C, true, w.ksum, w.vmax, k_mean, v_scale, w.vfac);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  QuantArgs a{};
+  a.kp = k; a.v = v; a.qp = q;
+  a.k_mean = k_mean; a.vfac = w.vfac;
+  a.k8 = k8; a.k_scale = k_scale; a.v8t = v8t;
+  a.B = B; a.Nq = N; a.Nkv = N; a.Hq = Hq; a.Hkv = Hkv;
+  a.G = 4 * ((N + 127) / 128);
+  a.nK = nK;
+  a.nq_blocks = 0;
+  a.k_rows = kKvRows;
+  a.nK_scale = nK;
+  a.nk_blocks = B * Hkv * nK;
+  a.nv_blocks = B * Hkv * nK;
+  a.k_raw = true; a.kw = kw; a.eps = eps; a.rotary_dim = rotary_dim; a.cos_t = cos_t; a.sin_t = sin_t;
+  const unsigned g2 = static_cast<unsigned>(a.nk_blocks + a.nv_blocks);
+  switch (D) {
+    case 64: quant_kernel<64><<<g2, 128, 0, st>>>(a); break;
+    case 128: quant_kernel<128><<<g2, 128, 0, st>>>(a); break;
+    case 256: quant_kernel<256><<<g2, 128, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Rotated INT8 Q only (q8 [B,Hq,Nq,D], one scale per 32-row group), or rotated
+// per-token INT8 K only, written at rows key0 .. key0+Nkv-1 of [B,Hkv,kcap,D]
+// (scales [B,Hkv,kcap]): the pieces of the chunked key-cache path.
+cudaError_t launch_hadamard_part(int B, int N, int H, int D, BNHD x, bool is_q, int8_t* x8,
+                                 void* scale, int kcap, int key0, cudaStream_t st) {
+  HadArgs a{};
+  a.B = B; a.Hq = H; a.Hkv = H; a.Nq = N; a.Nkv = N;
+  a.kcap = kcap; a.key0 = key0;
+  a.G = 4 * ((N + 127) / 128);
+  if (is_q) {
+    a.q = x; a.q8 = x8; a.q_scale = static_cast<float*>(scale);
+    a.nq_blocks = B * H * a.G;
+    a.nk_blocks = 0;
+  } else {
+    a.k = x; a.k8 = x8; a.k_scale16 = static_cast<uint16_t*>(scale);
+    a.nq_blocks = 0;
+    a.nk_blocks = static_cast<int>((static_cast<int64_t>(B) * H * N + 7) / 8);
+  }
+  const unsigned grid = static_cast<unsigned>(a.nq_blocks + a.nk_blocks);
+  switch (D) {
+    case 64: hadamard_quant_kernel<64><<<grid, 256, 0, st>>>(a); break;
+    case 256: hadamard_quant_kernel<256><<<grid, 256, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v16(int B, int n_src, int Hkv, int D, BNHD v, int cap, int key0,
+                             int n_write, uint16_t* v16t, cudaStream_t st) {
+  const dim3 grid((n_write + kKvRows - 1) / kKvRows, B * Hkv);
+  switch (D) {
+    case 64: quant_v16_kernel<64><<<grid, 128, 0, st>>>(v, n_src, Hkv, cap, key0, n_write, v16t); break;
+    case 128: quant_v16_kernel<128><<<grid, 128, 0, st>>>(v, n_src, Hkv, cap, key0, n_write, v16t); break;
+    case 256: quant_v16_kernel<256><<<grid, 128, 0, st>>>(v, n_src, Hkv, cap, key0, n_write, v16t); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -507,6 +870,7 @@ cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
   HadArgs a{};
   a.q = q; a.k = k; a.q8 = q8; a.q_scale = q_scale; a.k8 = k8; a.k_scale16 = k_scale16;
   a.B = B; a.Nq = Nq; a.Nkv = Nkv; a.Hq = Hq; a.Hkv = Hkv;
+  a.kcap = Nkv; a.key0 = 0;
   a.G = 4 * ((Nq + 127) / 128);
   a.nq_blocks = B * Hq * a.G;
   const int64_t toks = static_cast<int64_t>(B) * Hkv * Nkv;
@@ -521,7 +885,7 @@ cudaError_t launch_quant_hadamard(int B, int Nq, int Nkv, int Hq, int Hkv, int D
   if (e != cudaSuccess) return e;
   // V: per-channel FP8, same tiles as the standard quantizer (no Q, no K part)
   return launch_quant(B, Nq, Nkv, Hq, Hkv, D, q, k, v, nullptr, vfac, nullptr, nullptr, nullptr,
-                      nullptr, v8t, st);
+                      nullptr, v8t, st, kKvRows);
 }
 
 }  // namespace qattn

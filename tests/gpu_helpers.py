@@ -63,3 +63,35 @@ def oracle_full(w):
     if w.hadamard:
         return O.pipeline_hadamard(w.q, w.k, w.v)
     return O.pipeline(w.q, w.k, w.v, w.q_weight, w.k_weight, w.eps, w.rotary_dim, w.theta)
+
+
+SENTINEL = 0x7EADBEEF
+
+
+def hot_path_scores(pipe, tiles_list, sm_scale=0.0):
+    """INT32 score tiles of the quads in `tiles_list` as qattn_fwd's own kernel
+    computes them (qattn_scores: the mainloop's debug build), plus a check that
+    the attention output of that launch equals the pipeline's qattn_fwd output bit
+    for bit (the copy-out changes nothing else).  Slots start at a sentinel, so a
+    tile the kernel never reached shows up as a mismatch."""
+    tiles = torch.tensor(tiles_list, dtype=torch.int32, device=DEV)
+    s = torch.full((len(tiles_list), 128, 64), SENTINEL, dtype=torch.int32, device=DEV)
+    out = torch.empty_like(pipe.out)
+    qa.qattn_scores(pipe.B, pipe.Nq, pipe.Nkv, pipe.Hq, pipe.Hkv, pipe.D, pipe.q8, pipe.q_scale,
+                    pipe.k8, pipe.k_scale, 1 if pipe.hadamard else 0, pipe.v8t, pipe.v_scale,
+                    sm_scale, tiles, len(tiles_list), s, out, pipe.dev_err)
+    qa.qattn_check(pipe.dev_err)
+    assert torch.equal(out.view(torch.int16), pipe.out.view(torch.int16)), \
+        "the score copy-out build changed the attention output"
+    return host(s)
+
+
+def assert_scores_tile(got, q8_rows, k8_rows, what):
+    """got: one [128, 64] slot; q8_rows / k8_rows: the oracle's INT8 rows of that
+    query tile / key tile (fewer than 128 / 64 at a tail).  Valid entries equal
+    the integer dot products; rows past Nq and keys past Nkv read 0."""
+    from oracle import qattn_oracle as O
+    exp = O.scores(q8_rows, k8_rows)
+    nr, nc = exp.shape
+    assert np.array_equal(got[:nr, :nc], exp), what
+    assert not got[nr:].any() and not got[:, nc:].any(), f"{what}: tail not zero"

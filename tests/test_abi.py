@@ -21,8 +21,11 @@ def lib():
     return qa.load()
 
 
-def declared_functions():
-    src = open(HEADER).read()
+PROBE_HEADER = os.path.join(ROOT, "include", "qattn_probe.h")
+
+
+def declared_functions(path=HEADER):
+    src = open(path).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(qattn_\w+)\s*\(", src)))
 
@@ -30,10 +33,11 @@ def declared_functions():
 def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     assert set(names) == set(_lib.EXPORTED), names
+    assert set(declared_functions(PROBE_HEADER)) == set(_lib.EXPORTED_PROBE)
 
 
 def test_library_exports_every_declared_symbol(lib):
-    for name in declared_functions():
+    for name in declared_functions() + declared_functions(PROBE_HEADER):
         assert hasattr(lib, name), name
     assert lib.qattn_version().decode().startswith("qattn-b200")
 
@@ -61,7 +65,8 @@ def test_fwd_refusals(lib):
     assert call(Hq=3) == 4
     assert call(Nq=0) == 2
     assert call(B=-1) == 2
-    assert call(mode=2) == 4
+    assert call(mode=3) == 4
+    assert call(mode=-1) == 4
     assert call(sm_scale=-1.0) == 4
     assert call(sm_scale=float("nan")) == 4
     assert call(q8=None) == 1
@@ -114,8 +119,17 @@ def test_hadamard_needs_power_of_four_head_dim(lib):
 
 
 def test_scores_refusals(lib):
-    assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) == 2
-    assert lib.qattn_scores(1, 128, 128, 2, 2, 128, FAKE, FAKE, None, 4, FAKE, FAKE, None) == 1
+    def call(tiles=FAKE, n=4, s_out=FAKE, D=128, mode=0, out=FAKE):
+        return lib.qattn_scores(1, 128, 128, 2, 2, D, FAKE, FAKE, FAKE, FAKE, mode, FAKE, FAKE, 0.0,
+                                tiles, n, s_out, out, FAKE, None)
+    assert call(n=0) == 2
+    assert call(n=65537) == 2
+    assert call(tiles=None) == 1
+    assert call(s_out=None) == 1
+    assert call(tiles=FAKE + 4) == 3
+    assert call(D=96) == 4                 # then the qattn_fwd checks
+    assert call(mode=3) == 4
+    assert call(out=None) == 1
     assert lib.qattn_check(None, None) == 1
 
 
@@ -128,8 +142,8 @@ def test_stall_hook_refuses_negative_tiles_and_resets(lib):
 def test_host_pipeline_workspace_query_and_refusals(lib):
     ws = lib.qattn_host_workspace_bytes
     one = ws(1, 37810, 37810, 56, 56, 128, 7)
-    # two buffer sets, each at least the chunk's BF16 Q/K/V, prepared Q/K and output
-    assert one >= 2 * 6 * 37810 * 7 * 128 * 2
+    # two buffer sets, each at least the chunk's BF16 Q/K/V and output
+    assert one >= 2 * 4 * 37810 * 7 * 128 * 2
     assert ws(1, 37810, 37810, 56, 56, 128, 56) == ws(1, 37810, 37810, 56, 56, 128, 500)
     assert ws(1, 37810, 37810, 56, 56, 128, 8) > one
     assert ws(1, 100, 100, 4, 3, 128, 1) == 0        # Hq % Hkv
@@ -166,3 +180,39 @@ def test_default_host_chunk_rule():
     for args in [(1, 37810, 37810, 56, 56, 128), (2, 5000, 5000, 8, 2, 128), (1, 9000, 9000, 3, 3, 64)]:
         c = f(*args)
         assert 1 <= c <= args[4]
+
+
+def test_tc_probe_refusals(lib):
+    assert lib.qattn_tc_probe(2, 100, 148, FAKE, FAKE, None) == 2
+    assert lib.qattn_tc_probe(0, 0, 148, FAKE, FAKE, None) == 2
+    assert lib.qattn_tc_probe(0, (1 << 20) + 1, 148, FAKE, FAKE, None) == 2
+    assert lib.qattn_tc_probe(1, 100, 0, FAKE, FAKE, None) == 2
+    assert lib.qattn_tc_probe(1, 100, 148, None, FAKE, None) == 1
+    assert lib.qattn_tc_probe(1, 100, 148, FAKE, None, None) == 1
+
+
+def test_fp16_pv_refusals(lib):
+    def fwd(Nkv=128, cap=128, mode=1, v=FAKE):
+        return lib.qattn_fwd_pv16(1, 128, Nkv, 2, 2, 128, FAKE, FAKE, FAKE, FAKE, mode, v, cap, 0.0,
+                                  FAKE, FAKE, None)
+    assert fwd(cap=120) == 2                 # below Nkv
+    assert fwd(Nkv=100, cap=100) == 2        # not a multiple of 8
+    assert fwd(mode=3) == 4
+    assert fwd(v=None) == 1
+    assert fwd(v=FAKE + 8) == 3
+
+    def v16(N=100, cap=104, out=FAKE):
+        return lib.qattn_quant_v16(1, N, 2, 128, _view(), out, cap, None)
+    assert v16(cap=96) == 2
+    assert v16(cap=102) == 2
+    assert v16(out=None) == 1
+    assert v16(out=FAKE + 4) == 3
+    assert v16(N=0) == 2
+
+
+def test_quant_k32_refuses_like_quant(lib):
+    need = lib.qattn_quant_workspace_bytes(1, 64, 1, 128)
+    assert lib.qattn_quant_k32(1, 64, 64, 1, 1, 128, _view(), _view(), _view(), FAKE, FAKE, FAKE,
+                               FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == 5
+    assert lib.qattn_quant_k32(1, 64, 64, 1, 1, 96, _view(), _view(), _view(), FAKE, FAKE, FAKE,
+                               FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 4

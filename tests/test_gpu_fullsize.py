@@ -13,7 +13,7 @@ import quantized_exact_attention_qattn_b200 as qa
 from quantized_exact_attention_qattn_b200 import synth
 from oracle import qattn_oracle as O
 
-from gpu_helpers import DEV, assert_out_close, host, run_pipeline
+from gpu_helpers import assert_out_close, assert_scores_tile, host, hot_path_scores, run_pipeline
 
 pytestmark = pytest.mark.gpu
 
@@ -60,14 +60,11 @@ def test_canonical_prep_quant_bit_exact(canonical):
 
 
 def test_canonical_scores_bit_exact(canonical):
+    # the INT32 scores of qattn_fwd's own QK (the launch the benchmark times),
+    # query tiles {0, 147, 295 (50-row tail)} x key tiles {0, 295, 590 (50-key tail)}
     w, pipe = canonical
     tl = [(0, h, i, j) for h in SCORE_H for i in SCORE_Q for j in SCORE_K]
-    tiles = torch.tensor(tl, dtype=torch.int32, device=DEV)
-    s = torch.empty((len(tl), 128, 64), dtype=torch.int32, device=DEV)
-    qa.qattn_scores(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, pipe.q8, pipe.k8, tiles, len(tl), s,
-                    pipe.dev_err)
-    qa.qattn_check(pipe.dev_err)
-    s = host(s)
+    s = hot_path_scores(pipe, tl)
     # oracle INT8 operands of the sampled heads, from the inputs alone
     hs = list(SCORE_H)
     rows = _rows(w.Nq, SCORE_Q)
@@ -81,10 +78,7 @@ def test_canonical_scores_bit_exact(canonical):
         hi = hs.index(h)
         r0 = starts[i]
         nrows = min(128, w.Nq - 128 * i)
-        exp = O.scores(q8[b, hi, r0:r0 + nrows], k8[b, hi, 64 * j:64 * j + 64])
-        assert np.array_equal(s[n, :exp.shape[0], :exp.shape[1]], exp), (h, i, j)
-        # tail tiles: rows/keys past N read as zeros
-        assert not s[n, exp.shape[0]:].any() and not s[n, :, exp.shape[1]:].any()
+        assert_scores_tile(s[n], q8[b, hi, r0:r0 + nrows], k8[b, hi, 64 * j:64 * j + 64], (h, i, j))
 
 
 def test_canonical_output_sampled_rows(canonical):
@@ -110,3 +104,10 @@ def test_gqa_chunk_hadamard_full():
     for key in ("q8", "q_scale", "k8", "k_scale", "v8t", "v_scale"):
         assert np.array_equal(host(getattr(pipe, key)), ref[key]), key
     assert_out_close(host(pipe.out), ref["out"], "gqa_chunk")
+    # D = 256 split softmax (Q in tensor memory, QK overwriting S, integer-to-float
+    # conversion by the warps), GQA head mapping h -> h / 4, per-token K scales
+    tl = [(0, h, i, j) for h in (0, 5, 15) for i in (0, 7) for j in (0, 255, 511)]
+    s = hot_path_scores(pipe, tl)
+    for n, (b, h, i, j) in enumerate(tl):
+        assert_scores_tile(s[n], ref["q8"][b, h, 128 * i:128 * i + 128],
+                           ref["k8"][b, h // 4, 64 * j:64 * j + 64], (h, i, j))

@@ -1,7 +1,7 @@
 """GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
 
 Bit-exact: prepared Q/K, INT8 Q/K, their scales, the K mean, FP8 V and its
-scales, INT32 score tiles.  Tolerance (max-abs <= 2e-2, rel-L2 <= 5e-3): the
+scales, and the INT32 score tiles as the attention mainloop itself computes them.  Tolerance (max-abs <= 2e-2, rel-L2 <= 5e-3): the
 BF16 attention output."""
 import numpy as np
 import pytest
@@ -11,7 +11,8 @@ import quantized_exact_attention_qattn_b200 as qa
 from quantized_exact_attention_qattn_b200 import synth
 from oracle import qattn_oracle as O
 
-from gpu_helpers import (DEV, assert_out_close, dev_bf16, host, oracle_full, run_pipeline)
+from gpu_helpers import (DEV, SENTINEL, assert_out_close, assert_scores_tile, dev_bf16, host,
+                         hot_path_scores, oracle_full, run_pipeline)
 
 pytestmark = pytest.mark.gpu
 
@@ -41,18 +42,41 @@ def test_pipeline_parity(name):
 
 
 def test_scores_all_tiles_small():
+    # every tile of the small workload through the mainloop's own QK (Q in tensor
+    # memory, S accumulated onto the 1.5 * 2^23 preload), including the tail keys
     w = synth.make("small")
     pipe = run_pipeline(w)
     ref = oracle_full(w)
     nq, nk = O.ceil_div(w.Nq, 128), O.ceil_div(w.Nkv, 64)
     tl = [(0, h, i, j) for h in range(w.Hq) for i in range(nq) for j in range(nk)]
-    tiles = torch.tensor(tl, dtype=torch.int32, device=DEV)
-    s = torch.empty((len(tl), 128, 64), dtype=torch.int32, device=DEV)
-    qa.qattn_scores(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, pipe.q8, pipe.k8, tiles, len(tl), s,
-                    pipe.dev_err)
-    qa.qattn_check(pipe.dev_err)
-    s = host(s)
-    full = O.scores(ref["q8"], ref["k8"])          # [B,H,Nq,Nk]
+    s = hot_path_scores(pipe, tl)
     for n, (b, h, i, j) in enumerate(tl):
-        exp = full[b, h, 128 * i:128 * i + 128, 64 * j:64 * j + 64]
-        assert np.array_equal(s[n, :exp.shape[0], :exp.shape[1]], exp), (h, i, j)
+        assert_scores_tile(s[n], ref["q8"][b, h, 128 * i:128 * i + 128],
+                           ref["k8"][b, h, 64 * j:64 * j + 64], (h, i, j))
+
+
+def test_scores_encoder_d64_tails():
+    # D = 64 (Q in shared memory, three query tiles per CTA), B = 32: the last query
+    # tile has 89 rows, the last key tile 25 keys
+    w = synth.make("encoder")
+    pipe = run_pipeline(w)
+    nq, nk = O.ceil_div(w.Nq, 128), O.ceil_div(w.Nkv, 64)
+    tl = [(b, h, i, j) for b in (0, 31) for h in (0, 15) for i in (0, 2, nq - 1)
+          for j in (0, 5, nk - 1)]
+    s = hot_path_scores(pipe, tl)
+    q8, k8 = host(pipe.q8), host(pipe.k8)      # bit-exact against the oracle elsewhere
+    ref = oracle_full(w)
+    assert np.array_equal(q8, ref["q8"]) and np.array_equal(k8, ref["k8"])
+    for n, (b, h, i, j) in enumerate(tl):
+        assert_scores_tile(s[n], ref["q8"][b, h, 128 * i:128 * i + 128],
+                           ref["k8"][b, h, 64 * j:64 * j + 64], (b, h, i, j))
+
+
+def test_scores_requests_outside_the_problem_leave_slots_untouched():
+    w = synth.make("small")
+    pipe = run_pipeline(w)
+    tl = [(0, 0, 0, 0), (0, 5, 0, 0), (1, 0, 0, 0), (0, 0, 9, 0), (0, 0, 0, 99), (0, 0, 0, 0)]
+    s = hot_path_scores(pipe, tl)
+    assert np.array_equal(s[0], s[5])
+    for n in range(1, 5):
+        assert (s[n] == SENTINEL).all(), tl[n]

@@ -1,9 +1,10 @@
 """The allocation-free quantizer entry point.
 
 qattn_quant_noalloc serves callers that cannot allocate device memory while
-they quantize (inside a CUDA-graph capture, or under a memory manager that
-hands out only the tensors): its reduction scratch is a static device array
-inside the library.  It must give exactly what qattn_quant gives with a
+they quantize: an embedder whose memory manager owns all device memory and hands
+out only the tensors, or a runtime that must not allocate on its hot path because
+cudaMalloc and cudaFree can synchronize the device.  Its reduction scratch is a
+static device array inside the library.  It must give exactly what qattn_quant gives with a
 caller-provided workspace, on consecutive calls that reuse the same array, and
 refuse problems whose scratch would not fit.  This file is collected last so a
 stop-at-first-failure run has already run every other test.

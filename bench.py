@@ -89,12 +89,7 @@ def sum_over_ranks(x: float, dist, device=None) -> float:
     return float(t.item())
 
 
-def shard_heads(H: int, world: int, rank: int):
-    """Contiguous head range of `rank` when H heads are split over `world`
-    ranks (every head is an independent problem: no exchange is needed)."""
-    base, rem = divmod(H, world)
-    h0 = rank * base + min(rank, rem)
-    return h0, h0 + base + (1 if rank < rem else 0)
+from quantized_exact_attention_qattn_b200.shard import kv_shard, shard_heads  # noqa: E402,F401
 
 
 # ------------------------------------------------------------------ clocks
@@ -281,6 +276,44 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ side workloads
+def side_workloads(dev, reps: int = 20):
+    """Attention-call times of the pages' other workloads (not the benchmark
+    line's metric): the GQA prefill chunk with rotated int8 K (Nq1024 x Nkv32768,
+    16/4 heads, D256) and the 729-key encoder batch (B32 N729 H16 D64), each on
+    seeded device-generated inputs of the workload's shape, CUDA events, median."""
+    import torch
+    import quantized_exact_attention_qattn_b200 as qa
+    out = {}
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    for name, (B, Nq, Nkv, Hq, Hkv, D, had, rot) in {
+            "gqa_chunk": (1, 1024, 32768, 16, 4, 256, True, 0),
+            "encoder": (32, 729, 729, 16, 16, 64, False, 0)}.items():
+        q = torch.randn((B, Nq, Hq, D), device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn((B, Nkv, Hkv, D), device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn((B, Nkv, Hkv, D), device=dev, generator=g).to(torch.bfloat16)
+        pipe = qa.Pipeline(B, Nq, Nkv, Hq, Hkv, D, hadamard=had, device=dev)
+        w = (1 + 0.1 * torch.randn(D, device=dev, generator=g)).to(torch.bfloat16)
+        pipe.run(q, k, v, w, w, 1e-5, rot)
+        for _ in range(3):
+            pipe.run_fwd()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            pipe.run_fwd()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        pipe.check()
+        ms = percentile(ts, 0.5)
+        out[name] = {"fwd_ms": ms, "tflops": pipe.attn_ops / (ms / 1e3) / 1e12,
+                     "shape": {"B": B, "Nq": Nq, "Nkv": Nkv, "Hq": Hq, "Hkv": Hkv, "D": D,
+                               "rotated_int8_k": had}}
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args):
     import torch
@@ -293,10 +326,23 @@ def run_gpu(args):
     dist = init_dist(world, "nccl")
 
     w = make_workload(args.config)
+    import numpy as np
+    if args.shard_heads and world > 1:
+        # one problem split over the ranks by heads: each rank holds the column
+        # slice of the inputs with its heads (no exchange is needed anywhere)
+        (h0, h1), (k0, k1) = kv_shard(w.Hq, w.Hkv, world, rank)
+        if w.qkv is not None:
+            full = w.qkv.reshape(w.B, w.Nq, 3, w.Hq, w.D)
+            w.qkv = np.ascontiguousarray(full[:, :, :, h0:h1]).reshape(w.B * w.Nq, -1)
+            w.q = w.k = w.v = None
+        else:
+            w.q = np.ascontiguousarray(w.q[:, :, h0:h1])
+            w.k = np.ascontiguousarray(w.k[:, :, k0:k1])
+            w.v = np.ascontiguousarray(w.v[:, :, k0:k1])
+        w.Hq, w.Hkv = h1 - h0, k1 - k0
     if w.qkv is not None:
         host_qkv = torch.from_numpy(w.qkv).view(torch.bfloat16).pin_memory()
     else:   # contiguous workloads: one pinned buffer holding q | k | v
-        import numpy as np
         host_qkv = torch.from_numpy(np.concatenate([w.q.ravel(), w.k.ravel(), w.v.ravel()])
                                     ).view(torch.bfloat16).pin_memory()
     qkv = host_qkv.to(dev)
@@ -444,9 +490,14 @@ def run_gpu(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if (args.shard_heads and world > 1) else "weak",
+            "vs_baseline": None,
             "dtype": "int8 QK / e4m3 PV (f32 accumulate), bf16 in/out", "data": "synthetic",
-            "config": dict(workload_config(w), parallelism=f"{world} independent problems (one per GPU)"),
+            "config": dict(workload_config(w),
+                           parallelism=(f"one problem, heads split over {world} GPUs (no exchange)"
+                                        if (args.shard_heads and world > 1) else
+                                        f"{world} independent problems (one per GPU)")),
             "fwd_ms_per_call": fwd_ms,
             "fwd_ms_p10": percentile(fwd_all, 0.1),
             "fwd_ms_p90": percentile(fwd_all, 0.9),
@@ -479,6 +530,8 @@ def run_gpu(args):
         }
         if world == 1 and not args.no_cpu_baseline and args.config == "canonical":
             line["cpu_baseline"] = cpu_baseline_line(w)
+        if world == 1 and args.config == "canonical" and not args.no_side:
+            line["side_workloads"] = side_workloads(dev)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -495,6 +548,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-probe", action="store_true", help="skip the tensor-core peak probe")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side timings of the GQA-chunk and encoder attention calls")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="with N > 1 ranks: split one problem's heads over the ranks "
+                         "(strong scaling) instead of one whole problem per rank")
     ap.add_argument("--e2e-chunk", type=int, default=None,
                     help="KV heads per chunk of the end-to-end call (default Hkv // 8)")
     ap.add_argument("--config", default="canonical",

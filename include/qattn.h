@@ -244,9 +244,10 @@ qattn_status qattn_fwd(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  *                KV head) are kv_capacity apart: k8 [B,Hkv,kv_capacity,D],
  *                k_scale mode 0 [B,Hkv,ceil(cap/64)], mode 1 [B,Hkv,cap], mode 2
  *                [B,Hkv,ceil(cap/32)]; only the first Nkv keys are used
- *   v16t         FP16 [B,Hkv,D,kv_capacity] (device)
- *   kv_capacity  >= Nkv, a multiple of 8 (Nkv rounded up for a plain problem;
- *                the allocated length of a key cache)
+ *   v16t         FP16 [B,Hkv,D,vcap], vcap = kv_capacity rounded up to a multiple
+ *                of 8 (device; qattn_quant_v16 with capacity vcap)
+ *   kv_capacity  >= Nkv: Nkv for a plain problem, the allocated length of a key
+ *                cache
  * Errors: as qattn_fwd; SHAPE for kv_capacity. */
 qattn_status qattn_fwd_pv16(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
                             const int8_t* q8, const float* q_scale,

@@ -189,14 +189,15 @@ __device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
   }
 }
 
-// O <- O * o for the 64 O columns a thread owns in the two-threads-per-row layout
-// (16x32bx2 accesses: threads 0-15 columns 0-63 of their lanes, threads 16-31
-// columns 64-127), 32 columns at a time.
+// O <- O * o for the HALF O columns a thread owns in the two-threads-per-row
+// layout (16x32bx2 accesses: threads 0-15 columns 0 .. HALF-1 of their lanes,
+// threads 16-31 columns HALF .. 2 HALF-1), 32 columns at a time.
+template <int HALF>
 __device__ __forceinline__ void rescale_halves(uint32_t tO, float o) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < 64; c0 += 32) {
+  for (int c0 = 0; c0 < HALF; c0 += 32) {
     uint32_t r[32];
-    tmem_ld16x2_x32<64>(tO + c0, r);
+    tmem_ld16x2_x32<HALF>(tO + c0, r);
     tmem_wait_ld();
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
@@ -205,7 +206,7 @@ __device__ __forceinline__ void rescale_halves(uint32_t tO, float o) {
       r[j] = __float_as_uint(v.x);
       r[j + 1] = __float_as_uint(v.y);
     }
-    tmem_st16x2_x32<64>(tO + c0, r);
+    tmem_st16x2_x32<HALF>(tO + c0, r);
   }
 }
 

@@ -59,6 +59,9 @@ constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
 #ifndef QATTN_D128_HALVES
 #define QATTN_D128_HALVES 0
 #endif
+#ifndef QATTN_D256_HALVES
+#define QATTN_D256_HALVES 1
+#endif
 
 // PV 0: FP8 E4M3 P and V (kind::f8f6f4), two P buffers of 16 columns per query
 // tile; PV 1: FP16 P and V (kind::f16), one P buffer of 32 columns (the same
@@ -83,10 +86,14 @@ struct Cfg {
   // Softmax layout: one warpgroup per query tile owning whole 64-key rows, or (for
   // D = 256, where the longer P.V gives the softmax more time per tile and more
   // warps hide more of its latency) two per query tile, one per half of the keys.
-  static constexpr bool SPLIT = (D == 256);
-  // D = 128: two threads per query row inside one warp (16x32bx2 tensor-memory
-  // accesses), eight softmax warps per query tile, four per sub-partition in all
-  static constexpr bool HALVES = (D == 128) && (QATTN_D128_HALVES != 0);
+  // Two threads per query row inside one warp (16x32bx2 tensor-memory accesses),
+  // eight softmax warps per query tile
+  static constexpr bool HALVES = ((D == 128) && (QATTN_D128_HALVES != 0)) ||
+                                 ((D == 256) && (QATTN_D256_HALVES != 0));
+  static constexpr bool SPLIT = (D == 256) && !HALVES;
+  // D <= 128: S is preloaded with the bits of 1.5 * 2^23 and QK accumulates onto
+  // them; D = 256: QK overwrites S and the warps convert with I2F
+  static constexpr bool S_PRELOAD = (D <= 128);
   static constexpr int SM_WARPS = ((SPLIT || HALVES) ? 8 : 4) * NQT;  // softmax warps
   static constexpr int ARRIVALS = (SPLIT || HALVES) ? 8 : 4;          // softmax warps per query tile
   static constexpr int KS_PER_WARP = SPLIT ? 32 : 64;               // staged per-token K scales
@@ -269,8 +276,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          // split layout: the first K step overwrites S; full rows: onto the kMagic bits
-          const uint32_t acc = (C::SPLIT && kk == 0) ? 0u : 1u;
+          // D = 256: the first K step overwrites S; D <= 128: onto the kMagic bits
+          const uint32_t acc = (!C::S_PRELOAD && kk == 0) ? 0u : 1u;
           if constexpr (C::Q_TMEM)   // Q_i row r in lane r, 4 bytes per column, 8 columns per K step
             mma_i8_ts(tS, tmem + C::Q_COL + i * (D / 4) + kk * 8, bd, C::IDESC_QK, acc);
           else
@@ -599,14 +606,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         };
         float2 kpair_next = make_float2(0.0f, 0.0f);
         if constexpr (KMODE != 0) kpair_next = load_kpair(0);
-        {   // this thread's 64 bytes of its Q row into tensor memory (16 columns)
+        {   // this thread's D/2 bytes of its Q row into tensor memory (D/8 columns)
           const int n = qt * BM + row;
-          uint32_t r[16];
+          constexpr int QW = D / 8;                       // 32-bit words per thread
+          uint32_t r[QW];
           if (n < p.Nq) {
             const uint4* src = reinterpret_cast<const uint4*>(
-                p.q8 + (static_cast<int64_t>(bh) * p.Nq + n) * D + kh * 64);
+                p.q8 + (static_cast<int64_t>(bh) * p.Nq + n) * D + kh * (D / 2));
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < QW / 4; ++c) {
               const uint4 v = __ldg(src + c);
               r[4 * c] = v.x;
               r[4 * c + 1] = v.y;
@@ -615,14 +623,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) r[c] = 0u;
+            for (int c = 0; c < QW; ++c) r[c] = 0u;
           }
-          tmem_st16x2_x16<16>(tmem + lane_off + C::Q_COL + i * (D / 4), r);
+          if constexpr (QW == 16)
+            tmem_st16x2_x16<16>(tmem + lane_off + C::Q_COL + i * (D / 4), r);
+          else
+            tmem_st16x2_x32<32>(tmem + lane_off + C::Q_COL + i * (D / 4), r);
         }
-        // S accumulates onto the bits of kMagic (1.5 * 2^23), read back as FP32 it is
-        // exactly kMagic + S (|S| < 2^22)
-        tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);
-        tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
+        if constexpr (C::S_PRELOAD) {
+          // S accumulates onto the bits of kMagic (1.5 * 2^23), read back as FP32 it
+          // is exactly kMagic + S (|S| < 2^22)
+          tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);
+          tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -644,13 +657,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float x[32];                                    // keys 32 kh .. 32 kh + 31
           tmem_ld16x2_x32<32>(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
           tmem_wait_ld();
-          tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);     // reset S for QK_i(t+1)
-          tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
-          tmem_wait_st();
+          if constexpr (C::S_PRELOAD) {
+            tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);   // reset S for QK_i(t+1)
+            tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
+            tmem_wait_st();
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + i);
-          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kMagic);
+          if constexpr (!C::S_PRELOAD) {                  // INT32 scores to FP32: exact, |S| < 2^24
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
+          }
+          constexpr float kBias = C::S_PRELOAD ? kMagic : 0.0f;
+          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kBias);
           const bool last = (t == nK - 1);
           const int k0 = kh * 32;                         // first key of this half
           float mn;
@@ -670,14 +690,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
             float xmax = fmaxf(mq[0], mq[1]);
             xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 16));   // the row's other half
+            if constexpr (C::S_PRELOAD) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
-              x[j] = sj.x;
-              x[j + 1] = sj.y;
+              for (int j = 0; j < 32; j += 2) {
+                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+                x[j] = sj.x;
+                x[j + 1] = sj.y;
+              }
             }
             const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kBias), a);
             mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
             a2 = make_float2(a, a);
             nb2 = make_float2(-mn, -mn);
@@ -689,11 +711,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             kss[2 * lane] = kpair.x;
             kss[2 * lane + 1] = kpair.y;
             __syncwarp();
+            if constexpr (C::S_PRELOAD) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
-              x[j] = sj.x;
-              x[j + 1] = sj.y;
+              for (int j = 0; j < 32; j += 2) {
+                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+                x[j] = sj.x;
+                x[j + 1] = sj.y;
+              }
             }
             const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;
@@ -749,7 +773,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                                    abort, p.dev_err, kErrTimeoutO));
             if (!ok) break;
             tc_fence_after();
-            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_halves(tO, old);
+            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_halves<D / 2>(tO, old);
           }
           if constexpr (PV == 0)
             tmem_st16x2_x8<8>(tP + (t & 1) * (BN / 4), pk);   // keys 32 kh .. : columns 8 kh ..
@@ -770,12 +794,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           const float inv = rcp_approx(den);
           const int n = qt * BM + row;
-          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + kh * 64;
-          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + kh * 64;
+          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + kh * (D / 2);
+          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + kh * (D / 2);
 #pragma unroll 1
-          for (int c0 = 0; c0 < 64; c0 += 32) {
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
             uint32_t o[32];
-            tmem_ld16x2_x32<64>(tO + c0, o);
+            tmem_ld16x2_x32<D / 2>(tO + c0, o);
             tmem_wait_ld();
             if (n < p.Nq) {
               uint32_t w[16];
@@ -1046,11 +1070,11 @@ cudaError_t launch_fwd_t(const FwdLaunch& L, const ScoreDump& dump, cudaStream_t
   if (PV == 0)   // E4M3 [B,Hkv,D,64*nK]: rows past Nkv hold zeros
     ok = ok && make_map(&mV, L.v, static_cast<uint64_t>(nK) * BN, D, BH, BN, D,
                         CU_TENSOR_MAP_SWIZZLE_64B);
-  else           // FP16 [B,Hkv,D,kcap]: keys past Nkv read as zeros (outside the extent)
-    ok = ok && make_map_pitched(&mV, L.v, static_cast<uint64_t>(L.Nkv) * 2, D, BH,
-                                static_cast<uint64_t>(L.kcap) * 2,
-                                static_cast<uint64_t>(L.kcap) * 2 * D, BN * 2, D,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
+  else {         // FP16 [B,Hkv,D,vpitch]: keys past Nkv read as zeros (outside the extent)
+    const uint64_t vpitch = 8 * ((static_cast<uint64_t>(L.kcap) + 7) / 8);
+    ok = ok && make_map_pitched(&mV, L.v, static_cast<uint64_t>(L.Nkv) * 2, D, BH, vpitch * 2,
+                                vpitch * 2 * D, BN * 2, D, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (pointer alignment or size)";
     return cudaErrorInvalidValue;

@@ -260,9 +260,8 @@ static qattn_status fwd_common(int B, int Nq, int Nkv, int Hq, int Hkv, int D, c
   if (k_scale_mode < 0 || k_scale_mode > 2)
     return fail(QATTN_ERR_UNSUPPORTED,
                 "k_scale_mode %d (0: per 64 rows, 1: per token FP16, 2: per 32 rows)", k_scale_mode);
-  if (kcap < Nkv || (pv == 1 && kcap % 8 != 0))
-    return fail(QATTN_ERR_SHAPE, "%s: kv_capacity %d must be >= Nkv=%d%s", what, kcap, Nkv,
-                pv == 1 ? " and a multiple of 8" : "");
+  if (kcap < Nkv)
+    return fail(QATTN_ERR_SHAPE, "%s: kv_capacity %d must be >= Nkv=%d", what, kcap, Nkv);
   if (!(sm_scale >= 0.0f) || std::isinf(sm_scale))
     return fail(QATTN_ERR_UNSUPPORTED, "sm_scale must be finite and >= 0");
   QATTN_TRY(check_device());

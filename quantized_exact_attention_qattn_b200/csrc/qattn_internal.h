@@ -77,7 +77,8 @@ struct ScoreDump {
 // One attention launch.  k8 rows and k_scale entries per (batch, KV head) are
 // spaced kcap (>= Nkv) apart: kcap = Nkv for a plain problem, the allocated length
 // for a cache of which the first Nkv keys are used.  pv 0: v = E4M3
-// [B,Hkv,D,64*ceil(Nkv/64)] with v_scale; pv 1: v = FP16 [B,Hkv,D,kcap], no scale.
+// [B,Hkv,D,64*ceil(Nkv/64)] with v_scale; pv 1: v = FP16 [B,Hkv,D,kcap rounded up
+// to 8], no scale.
 // k_scale_mode 0: FP32 per 64 rows, 1: FP16 per token, 2: FP32 per 32 rows.
 struct FwdLaunch {
   int B, Nq, Nkv, Hq, Hkv, D;

@@ -181,8 +181,9 @@ struct QuantArgs {
   const uint16_t* sin_t;
 };
 
-// RoPE coefficients of the lane's 8 pairs at token n from the BF16 tables
-// [N][R/2] (R a multiple of 16, so the lane's 8 entries are one 16-byte chunk).
+// RoPE coefficients of the lane's 8 pairs at row n of BF16 tables [rows][R/2]
+// (R a multiple of 16, so the lane's 8 entries are one 16-byte chunk); the tables
+// may be in global or shared memory.
 __device__ __forceinline__ void table_coefs(const uint16_t* cos_t, const uint16_t* sin_t, int n,
                                             int half, int l, int half_lanes, float (&cv)[8],
                                             float (&sn)[8]) {
@@ -191,8 +192,24 @@ __device__ __forceinline__ void table_coefs(const uint16_t* cos_t, const uint16_
   unpack8(*reinterpret_cast<const uint4*>(sin_t + static_cast<int64_t>(n) * half + i0), sn);
 }
 
+// Copy the RoPE coefficients of tokens n0 .. n0+63 (clamped to N-1) from the
+// global tables [N][R/2] into shared memory [2][64][R/2] (all threads; the caller
+// synchronizes before use).
+__device__ __forceinline__ void stage_tables(const uint16_t* cos_t, const uint16_t* sin_t, int n0,
+                                             int N, int half, uint16_t* s_tab) {
+  const int per_tok = half / 8;                       // 16-byte chunks per token
+  for (int idx = threadIdx.x; idx < kKvRows * per_tok; idx += blockDim.x) {
+    const int tok = idx / per_tok, c = idx - tok * per_tok;
+    const int64_t n = min(n0 + tok, N - 1);
+    *reinterpret_cast<uint4*>(s_tab + tok * half + c * 8) =
+        *reinterpret_cast<const uint4*>(cos_t + n * half + c * 8);
+    *reinterpret_cast<uint4*>(s_tab + (kKvRows + tok) * half + c * 8) =
+        *reinterpret_cast<const uint4*>(sin_t + n * half + c * 8);
+  }
+}
+
 // RMSNorm + RoPE of one raw row chunk in the row layout of prep_row.cuh (L = D/8
-// lanes per row); `n` must index a valid table row (callers clamp it).
+// lanes per row); `n` indexes the row of the (global or staged) tables.
 template <int D>
 __device__ __forceinline__ uint4 prep_chunk(const uint4 raw, const uint16_t* w, float eps,
                                             int rotary_dim, const uint16_t* cos_t,
@@ -233,11 +250,18 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
                      : make_uint4(0, 0, 0, 0);
   }
   if (pa != nullptr) {
+    // the block's RoPE coefficients, staged once in shared memory (the row loads
+    // above are already in flight)
+    extern __shared__ __align__(16) uint16_t s_tab[];
+    const int half = pa->rotary_dim / 2;
+    if (half > 0) {
+      stage_tables(pa->cos_t, pa->sin_t, row0, N, half, s_tab);
+      __syncthreads();
+    }
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      const int n = row0 + (threadIdx.x + c * 128) / CPR;
-      raw[c] = prep_chunk<D>(raw[c], pa->kw, pa->eps, pa->rotary_dim, pa->cos_t, pa->sin_t,
-                             n < N ? n : 0);
+      const int r = (threadIdx.x + c * 128) / CPR;
+      raw[c] = prep_chunk<D>(raw[c], pa->kw, pa->eps, pa->rotary_dim, s_tab, s_tab + kKvRows * half, r);
     }
   }
   auto values = [&](int c, float (&x)[8]) {
@@ -388,46 +412,42 @@ struct PrepStatsArgs {
   double* ksum;                 // [B, nK, Hkv*D]
   float* vmax;                  // [B, nK, Hkv*D]
   int B, N, Hq, Hkv, G, nK;
+  int nq_ctas;                  // CTAs [0, nq_ctas) do Q, the rest K/V statistics
 };
 
-// First pass of the fused path, one CTA (256 threads) per (64-row block j, batch,
-// KV head): the block's rows of the KV head's Hq/Hkv query heads are prepared and
-// quantized at once (their two 32-row groups, "Q And K Quantization"); its K rows
-// are prepared and their FP64 column sums taken over the block in ascending row
-// order (the partials of the K mean, "Preparation" step 4); its V rows give the
-// block's column maxima of |v| ("V And PV").  Q leaves as INT8 with no BF16 copy;
-// K is prepared again from the raw rows by the quantizer's second pass.
+// First pass of the fused path, 128 threads per CTA, two kinds of CTA in one grid:
+//  * Q CTA (64-row block j, batch, query head): the block's rows are prepared and
+//    quantized at once, its two 32-row groups ("Q And K Quantization"); Q leaves
+//    as INT8 with no BF16 copy.
+//  * K/V CTA (64-row block j, batch, KV head): its K rows are prepared into shared
+//    memory and their FP64 column sums taken over the block in ascending row order
+//    (the partials of the K mean, "Preparation" step 4); its V rows give the
+//    block's column maxima of |v| ("V And PV").  K is prepared again from the raw
+//    rows by the second pass.
+// Both stage the block's 64 RoPE coefficient rows in shared memory once.
+// Dynamic shared memory: tables 2 x 64 x R/2 BF16, then (K/V CTAs) 64 x D BF16.
 template <int D>
-__global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) {
+__global__ void __launch_bounds__(128) prep_stats_kernel(const PrepStatsArgs a) {
   constexpr int L = D / 8, HPW = 32 / L;       // lanes per row, rows per warp
-  constexpr int RPP = 8 * HPW;                 // rows per pass (8 warps)
+  constexpr int RPP = 4 * HPW;                 // rows per pass (4 warps)
   constexpr int PASSES = kKvRows / RPP;
-  __shared__ float red[2][8];
-  __shared__ __align__(16) uint16_t sK[kKvRows * D];   // the block's prepared K rows
-  __shared__ unsigned vmx[D];                          // |v| column maxima (FP32 bits)
-  const int j = blockIdx.x;
-  const int bhk = blockIdx.y, b = bhk / a.Hkv, hk = bhk - b * a.Hkv;
+  extern __shared__ __align__(16) uint16_t dyn[];
+  __shared__ float red[2][4];
+  __shared__ unsigned vmx[D];                  // |v| column maxima (FP32 bits)
+  const int half = a.rotary_dim / 2;
+  uint16_t* s_tab = dyn;                       // [2][64][half]
+  uint16_t* sK = dyn + 2 * kKvRows * half;     // [64][D]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / L, l = lane - sub * L;
-  const int n0 = j * kKvRows;
-  const int nv = min(kKvRows, a.N - n0);              // valid rows of the block
-  const int Gh = a.Hq / a.Hkv;
-  if (threadIdx.x < D) vmx[threadIdx.x] = 0u;
   auto row_of = [&](int p) { return p * RPP + warp * HPW + sub; };
+  const bool is_q = static_cast<int>(blockIdx.x) < a.nq_ctas;
+  const int id = is_q ? blockIdx.x : blockIdx.x - a.nq_ctas;
+  const int j = id % a.nK;
+  const int bh = id / a.nK;                    // b * Hq + h (Q) or b * Hkv + hk (K/V)
+  const int n0 = j * kKvRows;
 
-  uint4 kraw[PASSES], vraw[PASSES];
-#pragma unroll
-  for (int p = 0; p < PASSES; ++p) {
-    const int n = n0 + row_of(p);
-    kraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.k, b, n, hk) + 8 * l)
-                      : make_uint4(0, 0, 0, 0);
-    vraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.v, b, n, hk) + 8 * l)
-                      : make_uint4(0, 0, 0, 0);
-  }
-
-  // ---- Q: prepare, group maxima, INT8 codes
-  for (int gi = 0; gi < Gh; ++gi) {
-    const int h = hk * Gh + gi;
+  if (is_q) {
+    const int h = bh % a.Hq, b = bh / a.Hq;
     uint4 y[PASSES];
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
@@ -435,11 +455,13 @@ __global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) 
       y[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.q, b, n, h) + 8 * l)
                      : make_uint4(0, 0, 0, 0);
     }
+    if (half > 0) stage_tables(a.cos_t, a.sin_t, n0, a.N, half, s_tab);
+    __syncthreads();
     float gmax[2] = {0.0f, 0.0f};
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
-      const int n = n0 + row_of(p);
-      y[p] = prep_chunk<D>(y[p], a.qw, a.eps, a.rotary_dim, a.cos_t, a.sin_t, n < a.N ? n : 0);
+      const int r = row_of(p), n = n0 + r;
+      y[p] = prep_chunk<D>(y[p], a.qw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half, r);
       if (n < a.N) {                                // rows past the end take no part
         float x[8];
         unpack8(y[p], x);
@@ -458,13 +480,10 @@ __global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) 
     float f[2];
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
-      float m = red[g][0];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[g][w]);
-      m = fmaxf(1e-7f, m);                          // a group with no row: 1e-7f
-      f[g] = __fdiv_rn(127.0f, m);
+      const float m = fmaxf(1e-7f, fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3])));
+      f[g] = __fdiv_rn(127.0f, m);                  // a group with no row: amax 1e-7f
       if (threadIdx.x == g)
-        a.q_scale[(static_cast<int64_t>(b) * a.Hq + h) * a.G + 2 * j + g] = __fdiv_rn(m, 127.0f);
+        a.q_scale[static_cast<int64_t>(bh) * a.G + 2 * j + g] = __fdiv_rn(m, 127.0f);
     }
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
@@ -479,27 +498,37 @@ __global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) 
         uint2 o;
         o.x = pack4_s8(q[0], q[1], q[2], q[3]);
         o.y = pack4_s8(q[4], q[5], q[6], q[7]);
-        *reinterpret_cast<uint2*>(a.q8 + ((static_cast<int64_t>(b) * a.Hq + h) * a.N + n) * D + 8 * l) = o;
+        *reinterpret_cast<uint2*>(a.q8 + (static_cast<int64_t>(bh) * a.N + n) * D + 8 * l) = o;
       }
     }
-    __syncthreads();                                // red is reused
-  }
-  // groups of the last 128-row tile past the last 64-row block hold no row
-  if (j == a.nK - 1) {
-    const int extra = a.G - 2 * a.nK;
-    for (int id = threadIdx.x; id < extra * Gh; id += blockDim.x) {
-      const int h = hk * Gh + id / extra, g = 2 * a.nK + id % extra;
-      a.q_scale[(static_cast<int64_t>(b) * a.Hq + h) * a.G + g] = __fdiv_rn(1e-7f, 127.0f);
+    // groups of the last 128-row tile past the last 64-row block hold no row
+    if (j == a.nK - 1) {
+      for (int g = 2 * a.nK + threadIdx.x; g < a.G; g += blockDim.x)
+        a.q_scale[static_cast<int64_t>(bh) * a.G + g] = __fdiv_rn(1e-7f, 127.0f);
     }
+    return;
   }
 
-  // ---- K: prepare into shared memory; V: column maxima
+  // ---- K/V statistics
+  const int hk = bh % a.Hkv, b = bh / a.Hkv;
+  const int nv = min(kKvRows, a.N - n0);              // valid rows of the block
+  uint4 kraw[PASSES], vraw[PASSES];
 #pragma unroll
   for (int p = 0; p < PASSES; ++p) {
-    const int r = row_of(p), n = n0 + r;
-    const uint4 y = prep_chunk<D>(kraw[p], a.kw, a.eps, a.rotary_dim, a.cos_t, a.sin_t,
-                                  n < a.N ? n : 0);
-    *reinterpret_cast<uint4*>(sK + r * D + 8 * l) = y;
+    const int n = n0 + row_of(p);
+    kraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.k, b, n, hk) + 8 * l)
+                      : make_uint4(0, 0, 0, 0);
+    vraw[p] = n < a.N ? *reinterpret_cast<const uint4*>(row_ptr(a.v, b, n, hk) + 8 * l)
+                      : make_uint4(0, 0, 0, 0);
+  }
+  for (int d = threadIdx.x; d < D; d += blockDim.x) vmx[d] = 0u;
+  if (half > 0) stage_tables(a.cos_t, a.sin_t, n0, a.N, half, s_tab);
+  __syncthreads();
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int r = row_of(p);
+    *reinterpret_cast<uint4*>(sK + r * D + 8 * l) =
+        prep_chunk<D>(kraw[p], a.kw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half, r);
   }
   float vm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
@@ -516,21 +545,21 @@ __global__ void __launch_bounds__(256) prep_stats_kernel(const PrepStatsArgs a) 
 #pragma unroll
     for (int off = L; off < 32; off <<= 1) vm[e] = fmaxf(vm[e], __shfl_xor_sync(0xffffffffu, vm[e], off));
   }
-  __syncthreads();                                  // vmx zeroed, sK written
   if (sub == 0) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) atomicMax(&vmx[8 * l + e], __float_as_uint(vm[e]));   // |v| >= 0
   }
+  __syncthreads();                                  // sK written, every atomicMax landed
   // FP64 column sums over the block's valid rows, ascending (one column per thread)
   const int C = a.Hkv * D;
   const size_t o = (static_cast<size_t>(b) * a.nK + j) * C + static_cast<size_t>(hk) * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    double s = 0.0;
-    for (int r = 0; r < nv; ++r) s = __dadd_rn(s, static_cast<double>(__uint_as_float(static_cast<uint32_t>(sK[r * D + d]) << 16)));
-    a.ksum[o + d] = s;
+    double sacc = 0.0;
+    for (int r = 0; r < nv; ++r)
+      sacc = __dadd_rn(sacc, static_cast<double>(__uint_as_float(static_cast<uint32_t>(sK[r * D + d]) << 16)));
+    a.ksum[o + d] = sacc;
+    a.vmax[o + d] = __uint_as_float(vmx[d]);
   }
-  __syncthreads();                                  // every atomicMax landed
-  for (int d = threadIdx.x; d < D; d += blockDim.x) a.vmax[o + d] = __uint_as_float(vmx[d]);
 }
 
 // ---------------------------------------------------------------- FP16 V
@@ -766,6 +795,19 @@ cudaError_t launch_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD qp
   return cudaGetLastError();
 }
 
+// Launch with `smem` bytes of dynamic shared memory (raising the kernel's limit
+// when it exceeds the default 48 KB).
+template <typename Args>
+cudaError_t launch_dyn(void (*kern)(const Args), unsigned grid, unsigned block, int smem,
+                       cudaStream_t st, const Args& a) {
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, block, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 size_t prep_quant_table_bytes(int N, int rotary_dim) {
   return ((static_cast<size_t>(N) * (rotary_dim / 2) * sizeof(uint16_t) + 255) & ~static_cast<size_t>(255)) * 2;
 }
@@ -787,15 +829,17 @@ cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   PrepStatsArgs pa{q, k, v, qw, kw, eps, rotary_dim, cos_t, sin_t, q8, q_scale, w.ksum, w.vmax,
-                   B, N, Hq, Hkv, 4 * ((N + 127) / 128), nK};
-  const dim3 grid(nK, B * Hkv);
+                   B, N, Hq, Hkv, 4 * ((N + 127) / 128), nK, nK * B * Hq};
+  const unsigned grid1 = static_cast<unsigned>(nK) * B * (Hq + Hkv);
+  const int tab_bytes = 2 * kKvRows * (rotary_dim / 2) * 2;
+  const int smem1 = tab_bytes + kKvRows * D * 2;
   switch (D) {
-    case 64: prep_stats_kernel<64><<<grid, 256, 0, st>>>(pa); break;
-    case 128: prep_stats_kernel<128><<<grid, 256, 0, st>>>(pa); break;
-    case 256: prep_stats_kernel<256><<<grid, 256, 0, st>>>(pa); break;
+    case 64: e = launch_dyn(prep_stats_kernel<64>, grid1, 128, smem1, st, pa); break;
+    case 128: e = launch_dyn(prep_stats_kernel<128>, grid1, 128, smem1, st, pa); break;
+    case 256: e = launch_dyn(prep_stats_kernel<256>, grid1, 128, smem1, st, pa); break;
     default: return cudaErrorInvalidValue;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (e != cudaSuccess) return e;
   const int C = Hkv * D;
   const int64_t cols = static_cast<int64_t>(B) * C;
   kv_finalize_kernel<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
@@ -815,13 +859,12 @@ cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD
   a.nv_blocks = B * Hkv * nK;
   a.k_raw = true; a.kw = kw; a.eps = eps; a.rotary_dim = rotary_dim; a.cos_t = cos_t; a.sin_t = sin_t;
   const unsigned g2 = static_cast<unsigned>(a.nk_blocks + a.nv_blocks);
-  switch (D) {
-    case 64: quant_kernel<64><<<g2, 128, 0, st>>>(a); break;
-    case 128: quant_kernel<128><<<g2, 128, 0, st>>>(a); break;
-    case 256: quant_kernel<256><<<g2, 128, 0, st>>>(a); break;
+  switch (D) {   // dynamic shared memory: the staged RoPE tables of a raw-K block
+    case 64: return launch_dyn(quant_kernel<64>, g2, 128, tab_bytes, st, a);
+    case 128: return launch_dyn(quant_kernel<128>, g2, 128, tab_bytes, st, a);
+    case 256: return launch_dyn(quant_kernel<256>, g2, 128, tab_bytes, st, a);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 // Rotated INT8 Q only (q8 [B,Hq,Nq,D], one scale per 32-row group), or rotated

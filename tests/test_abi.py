@@ -196,7 +196,6 @@ def test_fp16_pv_refusals(lib):
         return lib.qattn_fwd_pv16(1, 128, Nkv, 2, 2, 128, FAKE, FAKE, FAKE, FAKE, mode, v, cap, 0.0,
                                   FAKE, FAKE, None)
     assert fwd(cap=120) == 2                 # below Nkv
-    assert fwd(Nkv=100, cap=100) == 2        # not a multiple of 8
     assert fwd(mode=3) == 4
     assert fwd(v=None) == 1
     assert fwd(v=FAKE + 8) == 3

@@ -1,6 +1,7 @@
 """Multi-rank plumbing on CPU (gloo, world size 2): head sharding needs no
 exchange (each rank's heads give exactly the full-problem result for those
-heads), and the bench's max/sum-over-ranks timing reductions."""
+heads, also when each rank runs the whole path on its column slice of the raw
+interleaved QKV buffer), and the bench's max/sum-over-ranks timing reductions."""
 import os
 import socket
 
@@ -12,7 +13,7 @@ import torch.multiprocessing as mp
 
 import bench
 from oracle import qattn_oracle as O
-from quantized_exact_attention_qattn_b200 import synth
+from quantized_exact_attention_qattn_b200 import shard, synth
 
 
 def _free_port():
@@ -42,10 +43,27 @@ def _worker(rank, world, port, out_path):
                              v8t[:, h0:h1], vs[:, h0:h1], wk.Nkv)
     parts = [None] * world
     dist.all_gather_object(parts, (h0, h1, part))
+    # one interleaved problem split by heads at the raw input, as bench.py
+    # --shard-heads splits it: each rank runs the whole path (prep, K mean,
+    # quantization, attention) on the column slice of the QKV buffer holding its
+    # heads; gathered, every head equals the unsplit problem's
+    wc = synth.make("canonical", N=300, H=6)
+    (q0, q1), (k0, k1) = shard.kv_shard(wc.Hq, wc.Hkv, world, rank)
+    full5 = wc.qkv.reshape(1, wc.Nq, 3, wc.Hq, wc.D)
+    sl = [shard.head_slice(full5[:, :, i], a, b) for i, (a, b) in
+          enumerate([(q0, q1), (k0, k1), (k0, k1)])]
+    assert all(np.shares_memory(x, full5) for x in sl)      # views, no copy
+    mine = O.pipeline(sl[0], sl[1], sl[2], wc.q_weight, wc.k_weight, wc.eps, wc.rotary_dim,
+                      wc.theta)["out"]
+    raw_parts = [None] * world
+    dist.all_gather_object(raw_parts, (q0, mine))
     if rank == 0:
         full, _, _ = O.attention(q8, qs, k8, ks, v8t, vs, wk.Nkv)
         got = np.concatenate([p for _, _, p in sorted(parts, key=lambda x: x[0])], axis=2)
-        np.save(out_path, np.array([np.array_equal(got, full)]))
+        ref = O.pipeline(wc.q, wc.k, wc.v, wc.q_weight, wc.k_weight, wc.eps, wc.rotary_dim,
+                         wc.theta)["out"]
+        got2 = np.concatenate([p for _, p in sorted(raw_parts, key=lambda x: x[0])], axis=2)
+        np.save(out_path, np.array([np.array_equal(got, full) and np.array_equal(got2, ref)]))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -75,3 +93,11 @@ def test_percentile_nearest_rank():
     assert bench.percentile([7.0], 0.9) == 7.0
     ten = [float(i) for i in range(10)]
     assert bench.percentile(ten, 0.1) == 1.0 and bench.percentile(ten, 0.9) == 8.0
+
+
+@pytest.mark.parametrize("Hq,Hkv,world", [(16, 4, 2), (16, 4, 4), (56, 56, 8), (6, 3, 2)])
+def test_kv_shard_keeps_gqa_groups_whole(Hq, Hkv, world):
+    got = [shard.kv_shard(Hq, Hkv, world, r) for r in range(world)]
+    assert [h for (a, b), _ in got for h in range(a, b)] == list(range(Hq))
+    for (q0, q1), (k0, k1) in got:
+        assert all(h // (Hq // Hkv) in range(k0, k1) for h in range(q0, q1))

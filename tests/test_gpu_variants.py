@@ -32,7 +32,7 @@ def _pv16(pipe, v_dev, w, cap=None, mode=None):
     out = torch.empty((w.B, w.Nq, w.Hq, w.D), dtype=torch.bfloat16, device=DEV)
     mode = (1 if w.hadamard else 0) if mode is None else mode
     qa.qattn_fwd_pv16(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, pipe.q8, pipe.q_scale, pipe.k8,
-                      pipe.k_scale, mode, v16, cap, 0.0, out, pipe.dev_err)
+                      pipe.k_scale, mode, v16, w.Nkv, 0.0, out, pipe.dev_err)
     qa.qattn_check(pipe.dev_err)
     return host(v16).view(np.uint16), host(out)
 

@@ -255,6 +255,28 @@ qattn_status qattn_fwd_pv16(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
                             const uint16_t* v16t, int kv_capacity, float sm_scale,
                             uint16_t* out, int* dev_err, void* stream);
 
+/* Rotated INT8 V (page "npu plan P7", P7c: "an int8 V needs an inverse transform
+ * on the output that K does not").  qattn_quant_v_rotated:
+ *   v' = FWHT(v)/sqrt(D) per token (as qattn_quant_hadamard's K; D in {64, 256});
+ *   amax = max(1e-7f, max_n |v'|) per (b, h, channel); v_scale = amax/127.0f;
+ *   v8 = rni_sat_s8(v' * (127.0f/amax)), stored dim-major like the FP8 V:
+ *   v8t int8 [B,Hkv,D,64*ceil(Nkv/64)] (rows >= Nkv are 0), v_scale FP32 [B,Hkv,D]
+ *   workspace as qattn_quant (qattn_quant_workspace_bytes).
+ * qattn_fwd_int8v: qattn_fwd_pv16 with this V (D = 256): the INT8 tiles are
+ * widened exactly to FP16 on the chip (no FP16 copy of V in HBM), P16 . V8
+ * accumulates in FP32, and the output is rotated back:
+ *   o' = O * rcp(d) * v_scale (per rotated channel);  out = bf16_rn(FWHT(o')/sqrt(D)).
+ * Other arguments as qattn_fwd (k_scale_mode 0, 1 or 2).
+ * Errors: as qattn_fwd / qattn_quant; UNSUPPORTED for D. */
+qattn_status qattn_quant_v_rotated(int B, int Nkv, int Hkv, int D, qattn_bnhd v, int8_t* v8t,
+                                   float* v_scale, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+qattn_status qattn_fwd_int8v(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
+                             const int8_t* q8, const float* q_scale,
+                             const int8_t* k8, const void* k_scale, int k_scale_mode,
+                             const int8_t* v8t, const float* v_scale, float sm_scale,
+                             uint16_t* out, int* dev_err, void* stream);
+
 /* INT32 score tiles S = Q8 K8^T exactly as the attention mainloop computes them
  * ("INT8 QK And Score Domain"), for bit-exact checks of the path qattn_fwd runs.
  * This launches qattn_fwd's own kernel on the whole problem (same operands, same

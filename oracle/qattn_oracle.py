@@ -285,6 +285,28 @@ def quant_v16(v_bits: np.ndarray, capacity: int | None = None):
     return out
 
 
+def quant_v_rotated(v_bits: np.ndarray):
+    """INT8 V rotated by the per-head Walsh-Hadamard matrix (page "npu plan P7":
+    P7c, "an int8 V needs an inverse transform on the output that K does not").
+    Reading: V' = V H/sqrt(D) per token (the FP32 rotation of ``hadamard_rotate``),
+    INT8 with one scale per (batch, head, channel) over all tokens, the per-channel
+    maximum of "V And PV" with the INT8 formulas of "Q And K Quantization":
+    amax = max(1e-7f, max_n |v'|), v_scale = amax/127, v8 = rint_sat(v' * (127/amax)).
+    Returns v8t int8 [B,H,D,64*ceil(N/64)] (dim-major, keys contiguous, rows past N
+    are 0) and v_scale FP32 [B,H,D].
+    """
+    vr = hadamard_rotate(v_bits)                                # [B,N,H,D]
+    b, n, h, d = vr.shape
+    amax = np.maximum(AMAX_FLOOR, np.max(np.abs(vr), axis=1)).astype(F32)   # [B,H,D]
+    scale = (amax / F32(127.0)).astype(F32)
+    f = (F32(127.0) / amax).astype(F32)
+    codes = np.clip(np.rint((vr * f[:, None]).astype(F32)), -128, 127).astype(np.int8)
+    npad = KV_TILE * ceil_div(n, KV_TILE)
+    v8t = np.zeros((b, h, d, npad), dtype=np.int8)
+    v8t[:, :, :, :n] = codes.transpose(0, 2, 3, 1)
+    return v8t, scale
+
+
 # ============================================================ Hadamard variant
 def fwht(x: np.ndarray) -> np.ndarray:
     """Unnormalized Walsh-Hadamard transform along the last axis, FP32.
@@ -433,6 +455,13 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
       m     = mn
     out = bf16_rn((f32)(RO / d) * v_scale)      (reading: exact division)
 
+    pv="int8v" is the rotated INT8 V of the page "npu plan P7" (P7c): v8t holds the
+    INT8 codes of ``quant_v_rotated`` and v_scale its per-channel scales.  Reading:
+    probabilities as in pv="fp16" (P16 = fp16_rn(p)); RO += sum_j P16_j * V'8[j, :]
+    (exact tile sum); o' = (f32)(RO / d) * v_scale (FP32); the inverse rotation
+    out = bf16_rn(FWHT(o') / sqrt(D)) (H/sqrt(D) is symmetric and orthonormal, so
+    it is its own inverse; FP32 stages as ``fwht``, the 1/sqrt(D) scale exact).
+
     pv="fp16" is the FP16 P.V control of the page "Fused FP8 PV preparation"
     (softmax, maximum and denominator unchanged, only the probability encoding
     and V differ).  Reading: P16_j = fp16_rn(p_j), RO += sum_j P16_j * V16[j, :]
@@ -465,6 +494,8 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
         vv = f32_from_e4m3_bits(v8t).astype(np.float64)              # [B,Hkv,D,Np]
     elif pv == "fp16":
         vv = f32_from_f16_bits(v8t).astype(np.float64)
+    elif pv == "int8v":
+        vv = v8t.astype(np.float64)
     else:
         raise ValueError(pv)
     for t in range(nk):
@@ -507,9 +538,11 @@ def attention(q8, q_scale, k8, k_scale, v8t, v_scale, n_kv: int, *,
         ro = ro + np.matmul(pq.astype(np.float64), vt)
         m = mn
     o = (ro / den.astype(np.float64)[..., None]).astype(F32)
-    if pv == "fp8":
+    if pv in ("fp8", "int8v"):
         vs = v_scale[:, kvh].astype(F32)[:, :, None, :]
         o = (o * vs).astype(F32)
+    if pv == "int8v":
+        o = (fwht(o) * F32(1.0 / math.sqrt(d))).astype(F32)
     out = bf16_bits_from_f32(o).transpose(0, 2, 1, 3)                 # [B,R,Hq,D]
     return np.ascontiguousarray(out), m, den
 

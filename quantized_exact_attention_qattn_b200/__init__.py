@@ -14,13 +14,13 @@ from ._lib import (EXPORTED, QAttnError, bnhd, load, qattn_attention_host,  # no
                    qattn_prep, qattn_prep_quant, qattn_prep_quant_workspace_bytes, qattn_quant,
                    qattn_quant_hadamard, qattn_quant_noalloc, qattn_quant_workspace_bytes,
                    qattn_quant_k32, qattn_quant_v16, qattn_fwd_pv16, qattn_kcache_append,
-                   qattn_quant_q_hadamard,
+                   qattn_quant_q_hadamard, qattn_quant_v_rotated, qattn_fwd_int8v,
                    qattn_scores, qattn_tc_probe, qattn_version)
 
 __all__ = ["Pipeline", "HostRunner", "default_kv_heads_per_chunk", "QAttnError", "qattn_prep",
            "qattn_prep_quant", "qattn_prep_quant_workspace_bytes", "qattn_tc_probe", "qattn_quant",
            "qattn_quant_k32", "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append",
-           "qattn_quant_q_hadamard", "KCache",
+           "qattn_quant_q_hadamard", "qattn_quant_v_rotated", "qattn_fwd_int8v", "KCache",
            "qattn_quant_noalloc", "qattn_quant_hadamard",
            "qattn_fwd", "qattn_scores", "qattn_check", "qattn_quant_workspace_bytes",
            "qattn_host_workspace_bytes", "qattn_attention_host",

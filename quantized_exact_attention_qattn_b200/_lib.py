@@ -22,6 +22,7 @@ QATTN_STATUS = {0: "QATTN_OK", 1: "QATTN_ERR_NULL", 2: "QATTN_ERR_SHAPE", 3: "QA
 EXPORTED = ("qattn_prep", "qattn_quant_workspace_bytes", "qattn_quant", "qattn_quant_noalloc",
             "qattn_prep_quant_workspace_bytes", "qattn_prep_quant", "qattn_quant_k32",
             "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append", "qattn_quant_q_hadamard",
+            "qattn_quant_v_rotated", "qattn_fwd_int8v",
             "qattn_quant_hadamard",
             "qattn_fwd", "qattn_scores", "qattn_host_workspace_bytes", "qattn_attention_host",
             "qattn_check", "qattn_debug_stall_kv_tile", "qattn_last_error", "qattn_version")
@@ -64,11 +65,14 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_prep_quant_workspace_bytes.restype = sz
     lib.qattn_prep_quant.argtypes = [i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, f32, i, f64, i64, vp,
                                      vp, vp, vp, vp, vp, vp, vp, sz, vp]
-    lib.qattn_quant_k32.argtypes = lib.qattn_quant.argtypes
+    lib.qattn_quant_k32.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp, vp, vp,
+                                    vp, sz, vp]
     lib.qattn_quant_v16.argtypes = [i, i, i, i, BNHD, vp, i, vp]
     lib.qattn_fwd_pv16.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, i, f32, vp, vp, vp]
     lib.qattn_kcache_append.argtypes = [i, i, i, i, i, i, BNHD, BNHD, vp, vp, vp, vp]
     lib.qattn_quant_q_hadamard.argtypes = [i, i, i, i, BNHD, vp, vp, vp]
+    lib.qattn_quant_v_rotated.argtypes = [i, i, i, i, BNHD, vp, vp, vp, sz, vp]
+    lib.qattn_fwd_int8v.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, i, vp, vp, f32, vp, vp, vp]
     lib.qattn_quant_noalloc.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
                                         vp, vp, vp]
     lib.qattn_quant_hadamard.argtypes = [i, i, i, i, i, i, BNHD, BNHD, BNHD, vp, vp, vp, vp, vp,
@@ -87,7 +91,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qattn_version.restype = ctypes.c_char_p
     for name in ("qattn_prep", "qattn_prep_quant", "qattn_quant", "qattn_quant_noalloc",
                  "qattn_quant_k32", "qattn_quant_v16", "qattn_fwd_pv16", "qattn_kcache_append",
-                 "qattn_quant_q_hadamard", "qattn_quant_hadamard", "qattn_fwd",
+                 "qattn_quant_q_hadamard", "qattn_quant_v_rotated", "qattn_fwd_int8v", "qattn_quant_hadamard", "qattn_fwd",
                  "qattn_scores", "qattn_attention_host", "qattn_check", "qattn_debug_stall_kv_tile",
                  "qattn_tc_probe"):
         getattr(lib, name).restype = ctypes.c_int
@@ -186,6 +190,20 @@ def qattn_kcache_append(B, Hkv, D, n_new, key0, capacity, k, v, k8_cache, k_scal
 def qattn_quant_q_hadamard(B, Nq, Hq, D, q, q8, q_scale, stream=None):
     _check(load().qattn_quant_q_hadamard(B, Nq, Hq, D, bnhd(q), _ptr(q8), _ptr(q_scale),
                                          _stream(stream)))
+
+
+def qattn_quant_v_rotated(B, Nkv, Hkv, D, v, v8t, v_scale, workspace, workspace_bytes=None,
+                          stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().qattn_quant_v_rotated(B, Nkv, Hkv, D, bnhd(v), _ptr(v8t), _ptr(v_scale),
+                                        _ptr(workspace), nbytes, _stream(stream)))
+
+
+def qattn_fwd_int8v(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v8t, v_scale,
+                    sm_scale, out, dev_err, stream=None):
+    _check(load().qattn_fwd_int8v(B, Nq, Nkv, Hq, Hkv, D, _ptr(q8), _ptr(q_scale), _ptr(k8),
+                                  _ptr(k_scale), k_scale_mode, _ptr(v8t), _ptr(v_scale), sm_scale,
+                                  _ptr(out), _ptr(dev_err), _stream(stream)))
 
 
 def qattn_quant_noalloc(B, Nq, Nkv, Hq, Hkv, D, qp, kp, v, q8, q_scale, k8, k_scale, k_mean, v8t,

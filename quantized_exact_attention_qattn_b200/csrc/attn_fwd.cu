@@ -14,23 +14,23 @@
 //               kind::i8 (M=128, N=64, K=32 steps; for D >= 128 the Q tile is
 //               operand A in TMEM, stored there once by the softmax warps) into
 //               TMEM S[i] as soon as the softmax warps have read S[i], then P.V
-//               as kind::f8f6f4 with P read from TMEM (M=128, N=D, K=32)
-//               accumulating into TMEM O[i]
+//               (kind::f8f6f4 for FP8 P and V, kind::f16 for the FP16 variant) with
+//               P read from TMEM, accumulating into TMEM O[i]
 //   warps 4..   D <= 128: one 128-thread softmax warpgroup per query tile;
 //               thread r owns query row r (TMEM lane r): tcgen05.ld of its 64
-//               scores, the online-softmax update, tcgen05.st of its 64 FP8
+//               scores, the online-softmax update, tcgen05.st of its 64
 //               probabilities, the O rescale of its row (only in warps where some
 //               row's maximum moved, after the previous P.V completed), and the
 //               final normalisation + BF16 store.  S is preloaded with the bits
 //               of 1.5 * 2^23 and QK accumulates onto them, so the scores read
 //               back as FP32 with one packed subtract per pair and no conversion;
 //               the reader re-preloads S and releases it to the next QK at once.
-//   warps 3..   D = 256: two warpgroups per query tile, one per half of the 64
-//               keys (and of the O columns); the two warps on the same rows swap
-//               their half-row maxima through shared memory every tile, and add
-//               their partial denominators at the end.  Here QK overwrites S and
-//               the warps convert their 32 INT32 scores with I2F, which frees S
-//               for the next QK right after the load.
+//               D = 256: eight warps per query tile, two threads per row of the
+//               same warp (16x32bx2 accesses): each owns 32 of the tile's keys and
+//               half of the O columns, the row maximum is one shuffle between the
+//               two, and each keeps a partial denominator added at the end.  Here
+//               QK overwrites S and the warps convert their INT32 scores with I2F,
+//               which frees S for the next QK right after the load.
 // The query tiles' chains (two per CTA at D = 128, three at D = 64, where the
 // smaller O leaves TMEM room for a third) are independent, so while one warpgroup
 // runs the softmax of its tile the tensor core works for the others.  Every wait is
@@ -59,13 +59,13 @@ constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
 #ifndef QATTN_D128_HALVES
 #define QATTN_D128_HALVES 0
 #endif
-#ifndef QATTN_D256_HALVES
-#define QATTN_D256_HALVES 1
-#endif
 
 // PV 0: FP8 E4M3 P and V (kind::f8f6f4), two P buffers of 16 columns per query
 // tile; PV 1: FP16 P and V (kind::f16), one P buffer of 32 columns (the same
-// tensor-memory columns) and V tiles of 64 keys x 2 bytes per dim row.
+// tensor-memory columns) and V tiles of 64 keys x 2 bytes per dim row; PV 2 (D =
+// 256): as PV 1, with V arriving as rotated INT8 in a staging buffer that two
+// converter warps widen to the FP16 tile (exact), and the inverse rotation of the
+// output in the epilogue.
 template <int D, int NQT, int PV = 0>
 struct Cfg {
   static constexpr int STAGES = (D == 256) ? 3 : 4;
@@ -74,8 +74,9 @@ struct Cfg {
   static constexpr uint32_t SW_QK = (KCH == 128) ? 2u : 4u; // 128B or 64B swizzle
   static constexpr int Q_BYTES = BM * D;
   static constexpr int K_BYTES = BN * D;
-  static constexpr int VB = PV ? 2 : 1;                     // bytes per V element
+  static constexpr int VB = PV ? 2 : 1;                     // bytes per V element in the MMA tile
   static constexpr int V_BYTES = D * BN * VB;
+  static constexpr int VST_BYTES = (PV == 2) ? D * BN : 0;    // INT8 V staging (PV 2)
   // Q in tensor memory (A operand of QK read from TMEM, so each QK MMA reads only
   // its K tile from shared memory) wherever the columns allow: D = 128 with two
   // query tiles, D = 256 with one; D = 64 with three keeps Q in shared memory.
@@ -83,30 +84,24 @@ struct Cfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = SMEM_Q + (Q_TMEM ? 0 : NQT * Q_BYTES);
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
-  // Softmax layout: one warpgroup per query tile owning whole 64-key rows, or (for
-  // D = 256, where the longer P.V gives the softmax more time per tile and more
-  // warps hide more of its latency) two per query tile, one per half of the keys.
-  // Two threads per query row inside one warp (16x32bx2 tensor-memory accesses),
-  // eight softmax warps per query tile
-  static constexpr bool HALVES = ((D == 128) && (QATTN_D128_HALVES != 0)) ||
-                                 ((D == 256) && (QATTN_D256_HALVES != 0));
-  static constexpr bool SPLIT = (D == 256) && !HALVES;
+  // Softmax layout: one thread per query row (one warpgroup per query tile), or,
+  // for D = 256 (and D = 128 when QATTN_D128_HALVES is set), two threads per row
+  // inside one warp (16x32bx2 tensor-memory accesses), eight warps per query tile
+  static constexpr bool HALVES = (D == 256) || ((D == 128) && (QATTN_D128_HALVES != 0));
   // D <= 128: S is preloaded with the bits of 1.5 * 2^23 and QK accumulates onto
   // them; D = 256: QK overwrites S and the warps convert with I2F
   static constexpr bool S_PRELOAD = (D <= 128);
-  static constexpr int SM_WARPS = ((SPLIT || HALVES) ? 8 : 4) * NQT;  // softmax warps
-  static constexpr int ARRIVALS = (SPLIT || HALVES) ? 8 : 4;          // softmax warps per query tile
-  static constexpr int KS_PER_WARP = SPLIT ? 32 : 64;               // staged per-token K scales
-  static constexpr int SMEM_KS = SMEM_V + STAGES * V_BYTES;         // float [softmax warps][KS_PER_WARP]
-  static constexpr int SMEM_DEN = SMEM_KS + SM_WARPS * KS_PER_WARP * 4;  // float [NQT][2][128]
-  static constexpr int SMEM_PMAX = SMEM_DEN + NQT * 2 * BM * 4;     // float [NQT][2][2][128]
-  static constexpr int SMEM_BAR = SMEM_PMAX + NQT * 4 * BM * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 12 * NQT;
+  static constexpr int SM_WARPS = (HALVES ? 8 : 4) * NQT;           // softmax warps
+  static constexpr int ARRIVALS = HALVES ? 8 : 4;                   // softmax warps per query tile
+  static constexpr int SMEM_VST = SMEM_V + STAGES * V_BYTES;
+  static constexpr int SMEM_KS = SMEM_VST + STAGES * VST_BYTES;     // float [softmax warps][64]
+  static constexpr int SMEM_BAR = SMEM_KS + SM_WARPS * BN * 4;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 8 * NQT + (PV == 2 ? STAGES : 0);
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
   // warps 0..: producer, one MMA issuer per query tile (then a spare warp or two),
   // then the softmax warps; any four consecutive warps cover the four TMEM lane
   // quadrants (warp % 4)
-  static constexpr int SOFTMAX_WARP0 = SPLIT ? 3 : 4;
+  static constexpr int SOFTMAX_WARP0 = 4;
   static constexpr int THREADS = 32 * (SOFTMAX_WARP0 + SM_WARPS);
   // tensor memory columns: O[NQT] (D each), S[NQT] (64 each), P[NQT][2] (16 each)
   static constexpr uint32_t O_COL = 0;
@@ -155,8 +150,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token K scales
-  float* den_s = reinterpret_cast<float*>(smem + C::SMEM_DEN);     // partial denominators
-  float* pmax_s = reinterpret_cast<float*>(smem + C::SMEM_PMAX);   // half-row tile maxima
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
@@ -172,8 +165,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint64_t* p_full = s_free + NQT;           // [NQT][2] softmax -> MMA: P_i(t) written, O_i rescaled
   uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax: PV_i(t) done
   uint64_t* drain = pv_done + 2 * NQT;
-  uint64_t* pair_bar = drain + NQT;          // [NQT][4] the two halves of a row quadrant: tile maximum
-  uint64_t* q_ready = pair_bar + 4 * NQT;    // [NQT] softmax -> MMA: Q_i stored in tensor memory
+  uint64_t* q_ready = drain + NQT;           // [NQT] softmax -> MMA: Q_i stored in tensor memory
+  uint64_t* v_ready = q_ready + NQT;         // [STAGES] (PV 2) converters -> MMA: FP16 V tile written
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -205,10 +198,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(pv_done + 2 * i + bb, 1);
       }
       mbar_init(s_free + i, C::ARRIVALS);             // one lane per softmax warp
-      for (int q = 0; q < 4; ++q) mbar_init(pair_bar + i * 4 + q, 2);
       mbar_init(q_ready + i, C::ARRIVALS);            // one lane per softmax warp
     }
     for (int i = 0; i < NQT; ++i) mbar_init(drain + i, 1);
+    if constexpr (PV == 2)
+      for (int s = 0; s < C::STAGES; ++s) mbar_init(v_ready + s, 2);   // two converter warps
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -244,11 +238,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           issued = t + 1;
           continue;
         }
-        mbar_arrive_expect_tx(kv_full + s, static_cast<uint32_t>(C::K_BYTES + C::V_BYTES));
+        mbar_arrive_expect_tx(kv_full + s, static_cast<uint32_t>(C::K_BYTES + (PV == 2 ? C::VST_BYTES : C::V_BYTES)));
         for (int ch = 0; ch < C::NCH; ++ch)
           tma_load_3d(smem + C::SMEM_K + s * C::K_BYTES + ch * (BN * C::KCH), &tmK, kv_full + s,
                       ch * C::KCH, t * BN, bhkv);
-        tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN * C::VB, 0, bhkv);
+        if constexpr (PV == 2)   // INT8 tile into the staging buffer (unswizzled, 64 B rows)
+          tma_load_3d(smem + C::SMEM_VST + s * C::VST_BYTES, &tmV, kv_full + s, t * BN, 0, bhkv);
+        else
+          tma_load_3d(smem + C::SMEM_V + s * C::V_BYTES, &tmV, kv_full + s, t * BN * C::VB, 0, bhkv);
         issued = t + 1;
       }
       int dummy = 0;      // drain: every issued copy must land before the CTA may exit
@@ -315,6 +312,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mma_f8_ts(tO, a_tm + kk * 8, bd, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
           }
         } else {                   // one FP16 P buffer; V rows of 128 bytes, 128-byte swizzle
+          if constexpr (PV == 2) {  // the converter warps have written this stage's FP16 V
+            ok = mbar_wait(v_ready + s, (t / C::STAGES) & 1, abort, p.dev_err, kErrTimeoutKV);
+            if (!ok) break;
+            tc_fence_after();
+          }
           const uint32_t a_tm = tmem + C::P_COL + i * (BN / 2);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {   // K = 16 FP16 (32 bytes, 8 columns) per MMA
@@ -330,239 +332,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_wait(drain + i, 0, &dummy, p.dev_err, kErrTimeoutDrain);
     }
     __syncwarp();
-  } else if (warp >= C::SOFTMAX_WARP0) {
-    if constexpr (C::SPLIT) {
-      // ================================================================ softmax
-      // Two warpgroups per query tile i, one per half hf of the 64 key columns
-      // (warpgroup g = 2 i + hf).  Thread r of either owns query row r (TMEM lane r):
-      // both read all 64 scores for the tile maximum, each exponentiates, converts
-      // and stores its own 32, keeps its own partial denominator, and rescales and
-      // normalises its own half of the O columns.
-      const int g = (warp - C::SOFTMAX_WARP0) >> 2;
-      const int i = g >> 1, hf = g & 1;
-      const int q4 = warp & 3;
-      const int row = q4 * 32 + lane;
-      const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-      const uint32_t tO = tmem + lane_off + C::O_COL + i * D + hf * (D / 2);
-      bool ok = true;
-      float den = (hf == 0) ? 1.0f : 0.0f;   // the two halves' partial sums add up to d
-      if (i < nvalid) {
-        const int qt = qt0 + i;
-        const uint32_t tS = tmem + lane_off + C::S_COL + i * BN;
-        const uint32_t tS_own = tS + hf * 32;
-        // this half's 32 keys: 8 columns of P buffer (t & 1) (FP8) or 16 of the FP16 buffer
-        const uint32_t tP = tmem + lane_off + C::P_COL + i * (BN / 2) + hf * (PV ? BN / 4 : BN / 8);
-        const float qs = p.q_scale[static_cast<int64_t>(bh) * p.G + qt * 4 + q4];
-        const int last_valid = p.Nkv - (nK - 1) * BN;
-        const float* ks32 = static_cast<const float*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
-        const __half* ks16 = static_cast<const __half*>(p.k_scale) + static_cast<int64_t>(bhkv) * p.ks_stride;
-        const int n_groups32 = (p.Nkv + 31) / 32;        // scales per 32-row group (mode 2)
-        float m = kMInit;
-        float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
-        // per-key scales: lane l holds the scale of token 32 hf + l of a tile (0 past
-        // the end): its own (mode 1) or its 32-row group's (mode 2)
-        auto load_kone = [&](int tt) {
-          if constexpr (KMODE == 2) {
-            const int g = 2 * tt + hf;
-            return g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
-          } else {
-            const int j = tt * BN + hf * 32 + lane;
-            return j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f;
+  } else if (PV == 2 && warp < C::SOFTMAX_WARP0) {
+    // ================================================================ V converters (PV 2)
+    // Warps NQT+1 and NQT+2 widen each stage's INT8 V tile (dims x 64 keys,
+    // unswizzled) to the FP16 tile the P.V MMA reads (dims x 128 bytes, 128-byte
+    // swizzle: 16-byte chunk c of row d at c ^ (d & 7)), half of the dims each.
+    // b -> fp16: the bytes of (b ^ 0x80) under an exponent byte 0x64 are the FP16
+    // value 1024 + b + 128; subtracting 1152 leaves b exactly.
+    if constexpr (PV == 2) {
+      const int cw = warp - (NQT + 1);
+      const __half2 k1152 = __half2half2(__ushort_as_half(0x6480));
+      for (int t = 0; t < nK; ++t) {
+        const int s = t % C::STAGES;
+        if (!__all_sync(0xffffffffu, mbar_wait(kv_full + s, (t / C::STAGES) & 1, abort, p.dev_err,
+                                                kErrTimeoutKV)))
+          break;
+        const uint8_t* src = smem + C::SMEM_VST + s * C::VST_BYTES;
+        uint8_t* dst = smem + C::SMEM_V + s * C::V_BYTES;
+#pragma unroll 4
+        for (int k = 0; k < (D / 2) * 8 / 32; ++k) {
+          const int id = lane + 32 * k;
+          const int d = cw * (D / 2) + (id >> 3), c = id & 7;
+          const uint2 w = *reinterpret_cast<const uint2*>(src + d * BN + c * 8);
+          uint32_t o[4];
+          const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;
+          const uint32_t raw[4] = {__byte_perm(u0, 0x64646464u, 0x4140), __byte_perm(u0, 0x64646464u, 0x4342),
+                                   __byte_perm(u1, 0x64646464u, 0x4140), __byte_perm(u1, 0x64646464u, 0x4342)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __half2 hv = __hsub2(*reinterpret_cast<const __half2*>(&raw[q]), k1152);
+            o[q] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-        };
-        float kone_next = 0.0f;
-        if constexpr (KMODE != 0) kone_next = load_kone(0);
-        if constexpr (C::Q_TMEM) {   // this warp's rows, its half of the D bytes
-          store_q_row(p, bh, qt * BM + row, D, hf * 128, tmem + lane_off + C::Q_COL + i * (D / 4) + hf * 32);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(q_ready + i);
+          *reinterpret_cast<uint4*>(dst + d * (BN * 2) + ((c ^ (d & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        // s_free phase t: QK_i(t) may overwrite S_i (phase 0 needs nothing read)
-        if (lane == 0) mbar_arrive(s_free + i);
-        for (int t = 0; ok && t < nK; ++t) {
-          const float ks_cur = ks_next;
-          if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
-          const float kone = kone_next;
-          if constexpr (KMODE != 0) {
-            if (t + 1 < nK) kone_next = load_kone(t + 1);
-          }
-          ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, t & 1, abort, p.dev_err, kErrTimeoutS));
-          if (!ok) break;
-          tc_fence_after();
-          float x[32];                                    // this half's 32 scores
-          tmem_ld32(tS_own, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_free + i);         // S_i(t) read: QK_i(t+1) may overwrite it
-          // INT32 scores to FP32: exact, |S| <= D * 127^2 < 2^24
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
-          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, hf * 32, x, 0.0f);
-          const bool last = (t == nK - 1);
-          const int nv = last ? last_valid : BN;          // valid keys in this tile
-          const int own0 = hf * 32;                       // first key of this half
-          // The row's maximum over both halves: exchanged with the partner warp (same
-          // rows, other half) through shared memory, one slot per tile parity, behind a
-          // two-arrival mbarrier (a bounded wait).  Both warps then hold the same
-          // maximum, so both compute the same mn and old.
-          float* my_max = pmax_s + ((i * 2 + (t & 1)) * 2 + hf) * BM + row;
-          const float* their_max = pmax_s + ((i * 2 + (t & 1)) * 2 + (1 - hf)) * BM + row;
-          bool pair_ok = true;
-          auto pair_max = [&](float v) {
-            *my_max = v;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pair_bar + i * 4 + q4);
-            pair_ok = __all_sync(0xffffffffu, mbar_wait(pair_bar + i * 4 + q4, t & 1, abort, p.dev_err,
-                                                        kErrTimeoutS));
-            return fmaxf(v, *their_max);
-          };
-          float mn;
-          float2 a2, nb2;
-          if constexpr (KMODE == 0) {
-            // A = (q_scale * k_scale) * c; tile max of S*A from the max of S (A > 0)
-            if (last) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (own0 + j >= nv) x[j] = -INFINITY;     // masked key: p = 2^-inf = 0
-            }
-            // two independent chains over 16 values each: 7 three-input maxima + 1
-            float mq[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              mq[q] = fmaxf(x[16 * q], x[16 * q + 15]);
-#pragma unroll
-              for (int j = 1; j < 15; j += 2) mq[q] = fmax3(mq[q], x[16 * q + j], x[16 * q + j + 1]);
-            }
-            const float xmax = pair_max(fmaxf(mq[0], mq[1]));
-            if (!pair_ok) {
-              ok = false;
-              break;
-            }
-            const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-            const float smax = __fmul_rn(xmax, a);
-            mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
-            a2 = make_float2(a, a);
-            nb2 = make_float2(-mn, -mn);
-          } else {
-            // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
-            // fma(S_j, A_j, -mn).  The warp stages its half's 32 scales in shared
-            // memory (one per lane); every lane reads them all (broadcasts).
-            float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * 32;
-            kss[lane] = kone;                             // this tile's scale, fetched a tile ago
-            __syncwarp();
-            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
-            float smx = -INFINITY;
-            if (!last) {
-              smx = kt_tile_max<32>(x, kss, qs2, c2);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (own0 + j < nv)
-                  smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[j]), p.c)));
-            }
-            mn = fmaxf(m, __fsub_rn(pair_max(smx), kFp8Offset));
-            if (!pair_ok) {
-              ok = false;
-              break;
-            }
-            nb2 = make_float2(-mn, -mn);
-          }
-          const float old = ex2_approx(__fsub_rn(m, mn));
-          if constexpr (KMODE == 0) {
-            exp_block<0, 32>(x, a2, nb2);
-          } else {
-            exp_block_kt<0, 32>(x, ks_stage + (warp - C::SOFTMAX_WARP0) * 32, make_float2(qs, qs),
-                                make_float2(p.c, p.c), nb2);
-            __syncwarp();                                 // kss is rewritten next tile
-            if (last) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (own0 + j >= nv) x[j] = 0.0f;          // masked key: p = 0
-            }
-          }
-          // partial denominator: unquantized probabilities, four independent pair sums
-          float2 acc[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[q] = make_float2(x[2 * q], x[2 * q + 1]);
-#pragma unroll
-          for (int j = 8; j < 32; j += 8) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] = fadd2(acc[q], make_float2(x[j + 2 * q], x[j + 2 * q + 1]));
-          }
-          acc[0] = fadd2(acc[0], acc[1]);
-          acc[2] = fadd2(acc[2], acc[3]);
-          acc[0] = fadd2(acc[0], acc[2]);
-          den = __fadd_rn(__fmul_rn(den, old), __fadd_rn(acc[0].x, acc[0].y));
-          uint32_t pk[PV ? 16 : 8];
-          if constexpr (PV == 0) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) pk[j / 4] = cvt_e4m3x4(x[j], x[j + 1], x[j + 2], x[j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) pk[j / 2] = cvt_f16x2(x[j], x[j + 1]);
-          }
-          if (t >= 1) {
-            // PV_i(t-1) was issued when both halves finished tile t-1 and has long
-            // completed.  Its completion frees P buffer (t & 1), last read by
-            // PV_i(t-2), and lets this warp rescale its rows and half of O_i by
-            // old before PV_i(t) accumulates (only if some row's maximum moved).
-            ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((t - 1) & 1), ((t - 1) >> 1) & 1,
-                                                   abort, p.dev_err, kErrTimeoutO));
-            if (!ok) break;
-            tc_fence_after();
-            if (__any_sync(0xffffffffu, old != 1.0f)) rescale_rows<D / 2>(tO, old);
-          }
-          if constexpr (PV == 0)
-            tmem_st8(tP + (t & 1) * (BN / 4), pk);
-          else
-            tmem_st16(tP, pk);                            // PV_i(t-1) has read P_i(t-1)
-          tmem_wait_st();                                 // P and any O rescale have landed
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(p_full + 2 * i + (t & 1));
-          m = mn;
-        }
-        if (ok)
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 2 * i + ((nK - 1) & 1), ((nK - 1) >> 1) & 1,
-                                                 abort, p.dev_err, kErrTimeoutO));
-        // ---- finalize: O * rcp(d) * v_scale -> BF16, valid rows only ("Finalization").
-        // The two halves exchange partial denominators; d = d_0 + d_1 on both.
-        den_s[(i * 2 + hf) * BM + row] = den;
-        const bool any_failed = named_bar_red_or(9 + i, 256, !ok);
-        if (!any_failed) {
-          tc_fence_after();
-          const float inv = rcp_approx(__fadd_rn(den_s[(i * 2) * BM + row], den_s[(i * 2 + 1) * BM + row]));
-          const int n = qt * BM + row;
-          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + hf * (D / 2);
-          uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + hf * (D / 2);
-#pragma unroll 1
-          for (int c0 = 0; c0 < D / 2; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
-            if (n < p.Nq) {
-              uint32_t w[16];
-#pragma unroll
-              for (int j = 0; j < 32; j += 2) {
-                float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
-                                 make_float2(inv, inv));
-                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
-                w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
-              }
-              uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-              d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-              d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
-            }
-          }
-        }
+        fence_proxy_async_smem();                   // generic writes -> the tensor core's reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(v_ready + s);
       }
-    } else if constexpr (C::HALVES) {
+    }
+  } else if (warp >= C::SOFTMAX_WARP0) {
+    if constexpr (C::HALVES) {
       // ================================================================ softmax, D = 128
       // Eight warps per query tile, two threads per row of the same warp.  Warp
       // slot s = 0..7 of tile i covers lanes 32 (s % 4) + 16 (s / 4) .. +15 (its
@@ -794,8 +603,53 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           const float inv = rcp_approx(den);
           const int n = qt * BM + row;
-          const float* vs = PV ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + kh * (D / 2);
+          const float* vs = PV == 1 ? nullptr : p.v_scale + static_cast<int64_t>(bhkv) * D + kh * (D / 2);
           uint16_t* dst = p.out + ((static_cast<int64_t>(b) * p.Nq + n) * p.Hq + h) * D + kh * (D / 2);
+          if constexpr (PV == 2) {
+            // rotated V: o' = O * rcp(d) * v_scale (per rotated channel), then the
+            // inverse rotation out = FWHT(o') / sqrt(D): stages h = 1 .. D/4 inside
+            // this thread's D/2 columns, the last (h = D/2) against the row's other
+            // thread, in the oracle's stage order
+            constexpr int HC = D / 2;
+            float o[HC];
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld16x2_x32<HC>(tO + c0, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                o[c0 + j] = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), inv), vs[c0 + j]);
+            }
+#pragma unroll
+            for (int hh = 1; hh < HC; hh <<= 1) {
+#pragma unroll
+              for (int k2 = 0; k2 < HC; ++k2) {
+                if ((k2 & hh) == 0) {
+                  const float a0 = o[k2], b0 = o[k2 + hh];
+                  o[k2] = __fadd_rn(a0, b0);
+                  o[k2 + hh] = __fsub_rn(a0, b0);
+                }
+              }
+            }
+            constexpr float kInvSqrtD = (D == 256) ? 0.0625f : 0.125f;   // exact
+#pragma unroll
+            for (int k2 = 0; k2 < HC; ++k2) {
+              const float other = __shfl_xor_sync(0xffffffffu, o[k2], 16);
+              o[k2] = __fmul_rn(kh == 0 ? __fadd_rn(o[k2], other) : __fsub_rn(other, o[k2]), kInvSqrtD);
+            }
+            if (n < p.Nq) {
+#pragma unroll
+              for (int c0 = 0; c0 < HC; c0 += 8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  w4[q] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[c0 + 2 * q]))) |
+                          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[c0 + 2 * q + 1]))) << 16);
+                *reinterpret_cast<uint4*>(dst + c0) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
+            }
+          } else {
 #pragma unroll 1
           for (int c0 = 0; c0 < D / 2; c0 += 32) {
             uint32_t o[32];
@@ -807,7 +661,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               for (int j = 0; j < 32; j += 2) {
                 float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
                                  make_float2(inv, inv));
-                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                if constexpr (PV != 1) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
                 w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
                            (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
               }
@@ -817,6 +671,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
               d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
             }
+          }
           }
         }
       }
@@ -1029,7 +884,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               for (int j = 0; j < 32; j += 2) {
                 float2 v = fmul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])),
                                  make_float2(inv, inv));
-                if constexpr (PV == 0) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
+                if constexpr (PV != 1) v = fmul2(v, make_float2(vs[c0 + j], vs[c0 + j + 1]));
                 w[j / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
                            (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
               }
@@ -1070,6 +925,9 @@ cudaError_t launch_fwd_t(const FwdLaunch& L, const ScoreDump& dump, cudaStream_t
   if (PV == 0)   // E4M3 [B,Hkv,D,64*nK]: rows past Nkv hold zeros
     ok = ok && make_map(&mV, L.v, static_cast<uint64_t>(nK) * BN, D, BH, BN, D,
                         CU_TENSOR_MAP_SWIZZLE_64B);
+  else if (PV == 2)   // rotated INT8 [B,Hkv,D,64*nK] into the unswizzled staging buffer
+    ok = ok && make_map(&mV, L.v, static_cast<uint64_t>(nK) * BN, D, BH, BN, D,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
   else {         // FP16 [B,Hkv,D,vpitch]: keys past Nkv read as zeros (outside the extent)
     const uint64_t vpitch = 8 * ((static_cast<uint64_t>(L.kcap) + 7) / 8);
     ok = ok && make_map_pitched(&mV, L.v, static_cast<uint64_t>(L.Nkv) * 2, D, BH, vpitch * 2,
@@ -1105,6 +963,18 @@ template <int D, int NQT, int KMODE>
 cudaError_t launch_fwd_k(const FwdLaunch& L, const ScoreDump* dump, cudaStream_t st,
                          const char** why) {
   const ScoreDump none{nullptr, 0, nullptr};
+  if (L.pv == 2) {
+    if constexpr (D == 256) {
+      if (dump != nullptr) {
+        *why = "the score copy-out build exists for the FP8 P.V kernel only";
+        return cudaErrorInvalidValue;
+      }
+      return launch_fwd_t<D, NQT, KMODE, false, 2>(L, none, st, why);
+    } else {
+      *why = "rotated INT8 V needs D = 256";
+      return cudaErrorInvalidValue;
+    }
+  }
   if (L.pv == 1) {
     if (dump != nullptr) {
       *why = "the score copy-out build exists for the FP8 P.V kernel only";

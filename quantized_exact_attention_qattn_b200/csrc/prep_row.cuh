@@ -50,6 +50,64 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
+// Sum of squares of the row (L lanes of 8 consecutive dims, left to right, then
+// the XOR butterfly over the lanes): every lane of the row gets the same value.
+template <int D>
+__device__ __forceinline__ float sumsq8(const uint4 raw) {
+  constexpr int L = D / 8;
+  float x[8];
+  x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x);
+  x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
+  x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z);
+  x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
+  float ss = __fmul_rn(x[0], x[0]);
+#pragma unroll
+  for (int e = 1; e < 8; ++e) ss = __fadd_rn(ss, __fmul_rn(x[e], x[e]));
+#pragma unroll
+  for (int off = L / 2; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+  return ss;
+}
+
+// r = 1/sqrt(ss/D + eps), IEEE square root and division.
+template <int D>
+__device__ __forceinline__ float rms_r(float ss, float eps) {
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fmul_rn(ss, 1.0f / D), eps)));
+}
+
+// y = bf16(bf16(x * r) * w) for the lane's 8 values.
+__device__ __forceinline__ void apply_norm8(const uint4 raw, const uint16_t* w, float r, int l,
+                                            uint32_t (&yb)[4]) {
+  const uint4 wr = *reinterpret_cast<const uint4*>(w + 8 * l);
+  const uint32_t xv[4] = {raw.x, raw.y, raw.z, raw.w};
+  const uint32_t wv[4] = {wr.x, wr.y, wr.z, wr.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t xr = bf16x2_rn(fmul2(unpack_bf16x2(xv[j]), make_float2(r, r)));
+    yb[j] = bf16x2_rn(fmul2(unpack_bf16x2(xr), unpack_bf16x2(wv[j])));
+  }
+}
+
+// The r of N chunks' rows at once.  A warp holds 32/L rows per chunk; lane i <
+// N * (32/L) takes the sum of row (chunk i / (32/L), row i % (32/L)), computes its
+// r, and the values go back to the rows' lanes: one square root and division for
+// the warp's N * 32/L rows instead of one per chunk (the same bits).
+template <int D, int N>
+__device__ __forceinline__ void batch_rms_r(const float (&ss)[N], float eps, float (&r)[N]) {
+  constexpr int L = D / 8, HPW = 32 / L;
+  static_assert(N * HPW <= 32, "one lane per row");
+  const int lane = threadIdx.x & 31;
+  float mine = 0.0f;
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    const float t = __shfl_sync(0xffffffffu, ss[c], (lane % HPW) * L);
+    if (lane / HPW == c) mine = t;
+  }
+  const float rm = rms_r<D>(mine, eps);
+  const int sub = lane / L;
+#pragma unroll
+  for (int c = 0; c < N; ++c) r[c] = __shfl_sync(0xffffffffu, rm, c * HPW + sub);
+}
+
 // Step 1-2, RMSNorm: r = 1/sqrt(sum(x^2)/D + eps) with the sum taken as L lanes of
 // 8 consecutive dims (left to right) then an XOR butterfly over the lanes;
 // y = bf16(bf16(x * r) * w).  w == nullptr: no norm, y = x.  yb: the lane's 8

@@ -340,6 +340,40 @@ qattn_status qattn_fwd_pv16(int B, int Nq, int Nkv, int Hq, int Hkv, int D, cons
                     1, kv_capacity, sm_scale, out, dev_err, nullptr, stream, "qattn_fwd_pv16");
 }
 
+qattn_status qattn_fwd_int8v(int B, int Nq, int Nkv, int Hq, int Hkv, int D, const int8_t* q8,
+                             const float* q_scale, const int8_t* k8, const void* k_scale,
+                             int k_scale_mode, const int8_t* v8t, const float* v_scale,
+                             float sm_scale, uint16_t* out, int* dev_err, void* stream) {
+  if (D != 256)
+    return fail(QATTN_ERR_UNSUPPORTED, "qattn_fwd_int8v: rotated INT8 V needs D = 256, got %d", D);
+  return fwd_common(B, Nq, Nkv, Hq, Hkv, D, q8, q_scale, k8, k_scale, k_scale_mode, v8t, v_scale,
+                    2, Nkv, sm_scale, out, dev_err, nullptr, stream, "qattn_fwd_int8v");
+}
+
+qattn_status qattn_quant_v_rotated(int B, int Nkv, int Hkv, int D, qattn_bnhd v, int8_t* v8t,
+                                   float* v_scale, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  QATTN_TRY(check_sizes(B, Nkv, Nkv, Hkv, Hkv, D));
+  if (D != 64 && D != 256)
+    return fail(QATTN_ERR_UNSUPPORTED,
+                "Hadamard variant needs D in {64, 256} (1/sqrt(D) a power of two), got %d", D);
+  QATTN_TRY(check_view("v", v));
+  if (!v8t || !v_scale) return fail(QATTN_ERR_NULL, "quant_v_rotated: null output");
+  if (!aligned16(v8t)) return fail(QATTN_ERR_STRIDE, "quant_v_rotated: v8t must be 16-byte aligned");
+  if (workspace == nullptr || !aligned16(workspace))
+    return fail(QATTN_ERR_WORKSPACE, "quant_v_rotated: workspace is null or unaligned");
+  const size_t need = qattn::quant_workspace_bytes(B, Nkv, Hkv, D);
+  if (workspace_bytes < need)
+    return fail(QATTN_ERR_WORKSPACE, "quant_v_rotated: workspace of %zu bytes, %zu needed",
+                workspace_bytes, need);
+  QATTN_TRY(check_device());
+  qattn::QuantWorkspace w = qattn::carve_workspace(workspace, B, Nkv, Hkv, D);
+  cudaError_t e = qattn::launch_quant_v_rotated(B, Nkv, Hkv, D, qattn::to_bnhd(v), w, v8t, v_scale,
+                                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qattn_quant_v_rotated launch");
+  return QATTN_OK;
+}
+
 qattn_status qattn_quant_v16(int B, int Nkv, int Hkv, int D, qattn_bnhd v, uint16_t* v16t,
                              int capacity, void* stream) {
   QATTN_TRY(check_sizes(B, Nkv, Nkv, Hkv, Hkv, D));

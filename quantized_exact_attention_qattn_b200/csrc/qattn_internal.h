@@ -44,6 +44,10 @@ cudaError_t launch_quant(int B, int Nq, int Nkv, int Hq, int Hkv, int D, BNHD qp
                          BNHD v, const float* k_mean, const float* vfac, int8_t* q8,
                          float* q_scale, int8_t* k8, float* k_scale, uint8_t* v8t,
                          cudaStream_t st, int k_rows = 64);
+// Rotated INT8 V (V H/sqrt(D), per-channel scale amax/127), dim-major
+// [B, Hkv, D, 64*ceil(Nkv/64)]; uses ws.vmax / ws.vfac.
+cudaError_t launch_quant_v_rotated(int B, int Nkv, int Hkv, int D, BNHD v, QuantWorkspace ws,
+                                   int8_t* v8t, float* v_scale, cudaStream_t st);
 cudaError_t launch_hadamard_part(int B, int N, int H, int D, BNHD x, bool is_q, int8_t* x8,
                                  void* scale, int kcap, int key0, cudaStream_t st);
 // FP16 V, dim-major [B, Hkv, D, cap]: source rows -> keys key0 .. key0 + n_write

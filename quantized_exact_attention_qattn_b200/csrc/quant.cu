@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(256) kv_reduce_kernel(int Nkv, int Hkv, int D,
 // once to FP32; V maximum floored at 1e-7f, scale amax/2.25f and factor 2.25f/amax.
 __global__ void kv_finalize_kernel(int B, int Nkv, int nK, int C, bool has_k,
                                    const double* ksum, const float* vmax, float* k_mean,
-                                   float* v_scale, float* vfac) {
+                                   float* v_scale, float* vfac, float vrange = 2.25f) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<int64_t>(B) * C) return;
   const int b = static_cast<int>(idx / C), c = static_cast<int>(idx - static_cast<int64_t>(b) * C);
@@ -153,8 +153,8 @@ __global__ void kv_finalize_kernel(int B, int Nkv, int nK, int C, bool has_k,
   }
   if (has_k) k_mean[idx] = __double2float_rn(__ddiv_rn(s, static_cast<double>(Nkv)));
   a = fmaxf(1e-7f, a);
-  v_scale[idx] = __fdiv_rn(a, 2.25f);
-  vfac[idx] = __fdiv_rn(2.25f, a);
+  v_scale[idx] = __fdiv_rn(a, vrange);      // 2.25 for E4M3 V, 127 for rotated INT8 V
+  vfac[idx] = __fdiv_rn(vrange, a);
 }
 
 // ---------------------------------------------------------------- quantizer
@@ -208,6 +208,49 @@ __device__ __forceinline__ void stage_tables(const uint16_t* cos_t, const uint16
   }
 }
 
+// RoPE of one normalized row chunk (BF16 pairs yb) in the row layout of
+// prep_row.cuh; `n` indexes the row of the (global or staged) tables.
+template <int D>
+__device__ __forceinline__ uint4 rope_chunk(uint32_t (&yb)[4], int rotary_dim,
+                                            const uint16_t* cos_t, const uint16_t* sin_t, int n) {
+  constexpr int L = D / 8;
+  const int lane = threadIdx.x & 31, sub = lane / L, l = lane - sub * L;
+  const int rot_lanes = rotary_dim / 8, half = rotary_dim / 2, half_lanes = half / 8;
+  if (rot_lanes > 0) {
+    float cv[8], sn[8];
+    if (l < rot_lanes) table_coefs(cos_t, sin_t, n, half, l, half_lanes, cv, sn);
+    prep::rope8(yb, sub, l, L, half_lanes, rot_lanes, cv, sn);
+  }
+  return make_uint4(yb[0], yb[1], yb[2], yb[3]);
+}
+
+// RMSNorm + RoPE of N raw row chunks of a thread (chunk c: row `rows[c]` of the
+// tables), with the rows' r computed together (batch_rms_r).  w == nullptr: no norm.
+template <int D, int N>
+__device__ __forceinline__ void prep_chunks(uint4 (&x)[N], const int (&rows)[N], const uint16_t* w,
+                                            float eps, int rotary_dim, const uint16_t* cos_t,
+                                            const uint16_t* sin_t) {
+  constexpr int L = D / 8;
+  const int l = (threadIdx.x & 31) % L;
+  float r[N];
+  if (w != nullptr) {
+    float ss[N];
+#pragma unroll
+    for (int c = 0; c < N; ++c) ss[c] = prep::sumsq8<D>(x[c]);
+    prep::batch_rms_r<D, N>(ss, eps, r);
+  }
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    uint32_t yb[4];
+    if (w != nullptr) {
+      prep::apply_norm8(x[c], w, r[c], l, yb);
+    } else {
+      yb[0] = x[c].x; yb[1] = x[c].y; yb[2] = x[c].z; yb[3] = x[c].w;
+    }
+    x[c] = rope_chunk<D>(yb, rotary_dim, cos_t, sin_t, rows[c]);
+  }
+}
+
 // RMSNorm + RoPE of one raw row chunk in the row layout of prep_row.cuh (L = D/8
 // lanes per row); `n` indexes the row of the (global or staged) tables.
 template <int D>
@@ -258,11 +301,10 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
       stage_tables(pa->cos_t, pa->sin_t, row0, N, half, s_tab);
       __syncthreads();
     }
+    int rows[CH];
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int r = (threadIdx.x + c * 128) / CPR;
-      raw[c] = prep_chunk<D>(raw[c], pa->kw, pa->eps, pa->rotary_dim, s_tab, s_tab + kKvRows * half, r);
-    }
+    for (int c = 0; c < CH; ++c) rows[c] = (threadIdx.x + c * 128) / CPR;
+    prep_chunks<D, CH>(raw, rows, pa->kw, pa->eps, pa->rotary_dim, s_tab, s_tab + kKvRows * half);
   }
   auto values = [&](int c, float (&x)[8]) {
     const int id = threadIdx.x + c * 128;
@@ -306,7 +348,9 @@ __device__ __forceinline__ void quant_group(const BNHD& src, const float* mean, 
   }
 }
 
-template <int D>
+// KRAW: the fused path's second pass (K blocks prepared from raw rows); a separate
+// instance so the two-step quantizer keeps its own (smaller) register budget.
+template <int D, bool KRAW = false>
 __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
   __shared__ float red[4];
   __shared__ __align__(16) uint8_t tile[D * kKvRows];
@@ -324,12 +368,14 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
     const int h = bh % a.Hkv, b = bh / a.Hkv;
     const float* mean = a.k_mean + static_cast<int64_t>(bh) * D;
     float* sc = a.k_scale + static_cast<int64_t>(bh) * a.nK_scale + j;
-    if (a.k_rows == kKvRows)
-      quant_group<D, kKvRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kKvRows, a.k8, sc, red,
-                              a.k_raw ? &a : nullptr);
-    else
-      quant_group<D, kQRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kQRows, a.k8, sc, red,
-                             a.k_raw ? &a : nullptr);
+    if constexpr (KRAW) {
+      quant_group<D, kKvRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kKvRows, a.k8, sc, red, &a);
+    } else {
+      if (a.k_rows == kKvRows)
+        quant_group<D, kKvRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kKvRows, a.k8, sc, red);
+      else
+        quant_group<D, kQRows>(a.kp, mean, b, h, a.Hkv, a.Nkv, j * kQRows, a.k8, sc, red);
+    }
     return;
   }
   blk -= a.nk_blocks;
@@ -426,13 +472,16 @@ struct PrepStatsArgs {
 //    rows by the second pass.
 // Both stage the block's 64 RoPE coefficient rows in shared memory once.
 // Dynamic shared memory: tables 2 x 64 x R/2 BF16, then (K/V CTAs) 64 x D BF16.
+constexpr int kPrepStatsThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(128) prep_stats_kernel(const PrepStatsArgs a) {
+__global__ void __launch_bounds__(kPrepStatsThreads) prep_stats_kernel(const PrepStatsArgs a) {
   constexpr int L = D / 8, HPW = 32 / L;       // lanes per row, rows per warp
-  constexpr int RPP = 4 * HPW;                 // rows per pass (4 warps)
+  constexpr int NW = kPrepStatsThreads / 32;
+  constexpr int RPP = NW * HPW;                // rows per pass
   constexpr int PASSES = kKvRows / RPP;
   extern __shared__ __align__(16) uint16_t dyn[];
-  __shared__ float red[2][4];
+  __shared__ float red[2][NW];
   __shared__ unsigned vmx[D];                  // |v| column maxima (FP32 bits)
   const int half = a.rotary_dim / 2;
   uint16_t* s_tab = dyn;                       // [2][64][half]
@@ -457,11 +506,14 @@ __global__ void __launch_bounds__(128) prep_stats_kernel(const PrepStatsArgs a) 
     }
     if (half > 0) stage_tables(a.cos_t, a.sin_t, n0, a.N, half, s_tab);
     __syncthreads();
+    int rows[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) rows[p] = row_of(p);
+    prep_chunks<D, PASSES>(y, rows, a.qw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half);
     float gmax[2] = {0.0f, 0.0f};
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
-      const int r = row_of(p), n = n0 + r;
-      y[p] = prep_chunk<D>(y[p], a.qw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half, r);
+      const int n = n0 + row_of(p);
       if (n < a.N) {                                // rows past the end take no part
         float x[8];
         unpack8(y[p], x);
@@ -480,7 +532,10 @@ __global__ void __launch_bounds__(128) prep_stats_kernel(const PrepStatsArgs a) 
     float f[2];
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
-      const float m = fmaxf(1e-7f, fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3])));
+      float m = red[g][0];
+#pragma unroll
+      for (int w2 = 1; w2 < NW; ++w2) m = fmaxf(m, red[g][w2]);
+      m = fmaxf(1e-7f, m);
       f[g] = __fdiv_rn(127.0f, m);                  // a group with no row: amax 1e-7f
       if (threadIdx.x == g)
         a.q_scale[static_cast<int64_t>(bh) * a.G + 2 * j + g] = __fdiv_rn(m, 127.0f);
@@ -524,11 +579,14 @@ __global__ void __launch_bounds__(128) prep_stats_kernel(const PrepStatsArgs a) 
   for (int d = threadIdx.x; d < D; d += blockDim.x) vmx[d] = 0u;
   if (half > 0) stage_tables(a.cos_t, a.sin_t, n0, a.N, half, s_tab);
   __syncthreads();
+  {
+    int rows[PASSES];
 #pragma unroll
-  for (int p = 0; p < PASSES; ++p) {
-    const int r = row_of(p);
-    *reinterpret_cast<uint4*>(sK + r * D + 8 * l) =
-        prep_chunk<D>(kraw[p], a.kw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half, r);
+    for (int p = 0; p < PASSES; ++p) rows[p] = row_of(p);
+    prep_chunks<D, PASSES>(kraw, rows, a.kw, a.eps, a.rotary_dim, s_tab, s_tab + kKvRows * half);
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p)
+      *reinterpret_cast<uint4*>(sK + rows[p] * D + 8 * l) = kraw[p];
   }
   float vm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
@@ -730,7 +788,100 @@ __global__ void __launch_bounds__(256) hadamard_quant_kernel(const HadArgs a) {
   store_q8_e<D>(a.k8 + slot * D, v, f);
 }
 
+// ---------------------------------------------------------------- rotated INT8 V
+// V' = V H/sqrt(D) per token (fwht_row, the rotation of the K path), INT8 with one
+// scale per (batch, head, channel).  Statistics: one CTA (8 warps) per (64-row
+// block j, batch, head), a warp per row, |v'| column maxima of the block.
+template <int D>
+__global__ void __launch_bounds__(256) vrot_stats_kernel(BNHD v, int Nkv, int Hkv, int nK,
+                                                         float* vmax) {
+  constexpr int E = D / 32;
+  constexpr float kNorm = (D == 256) ? 0.0625f : 0.125f;   // 1/sqrt(D), exact
+  __shared__ unsigned cmax[D];
+  const int j = blockIdx.x, bh = blockIdx.y, b = bh / Hkv, h = bh - b * Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) cmax[d] = 0u;
+  __syncthreads();
+  float m[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) m[e] = 0.0f;
+  for (int r = warp; r < kKvRows; r += 8) {
+    const int n = j * kKvRows + r;
+    if (n >= Nkv) break;                             // warp-uniform
+    float x[E];
+    load_row_e<D>(v, b, n, h, x);
+    fwht_row<D>(x);
+#pragma unroll
+    for (int e = 0; e < E; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(x[e], kNorm)));
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) atomicMax(&cmax[lane * E + e], __float_as_uint(m[e]));
+  __syncthreads();
+  const size_t o = (static_cast<size_t>(b) * nK + j) * Hkv * D + static_cast<size_t>(h) * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) vmax[o + d] = __uint_as_float(cmax[d]);
+}
+
+// Codes: one CTA per (64-row block, batch, head): rows rotated again (the same
+// arithmetic), times 127/amax of their channel, rint-sat to INT8, transposed into
+// the dim-major [B, H, D, 64 nK] tile (keys past Nkv are 0).
+template <int D>
+__global__ void __launch_bounds__(256) vrot_quant_kernel(BNHD v, int Nkv, int Hkv, int nK,
+                                                         const float* vfac, int8_t* v8t) {
+  constexpr int E = D / 32;
+  constexpr float kNorm = (D == 256) ? 0.0625f : 0.125f;
+  __shared__ __align__(16) int8_t tile[D * kKvRows];   // [d][key]
+  const int j = blockIdx.x, bh = blockIdx.y, b = bh / Hkv, h = bh - b * Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* fac = vfac + static_cast<int64_t>(bh) * D;
+  float f[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) f[e] = fac[lane * E + e];
+  for (int r = warp; r < kKvRows; r += 8) {
+    const int n = j * kKvRows + r;
+    float x[E];
+    if (n < Nkv) {
+      load_row_e<D>(v, b, n, h, x);
+      fwht_row<D>(x);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      tile[(lane * E + e) * kKvRows + r] = n < Nkv ? q8_of(__fmul_rn(__fmul_rn(x[e], kNorm), f[e])) : 0;
+  }
+  __syncthreads();
+  const int64_t npad = static_cast<int64_t>(nK) * kKvRows;
+  int8_t* dst = v8t + static_cast<int64_t>(bh) * D * npad + static_cast<int64_t>(j) * kKvRows;
+  for (int id = threadIdx.x; id < D * (kKvRows / 16); id += blockDim.x) {
+    const int d = id / (kKvRows / 16), c = id - d * (kKvRows / 16);
+    *reinterpret_cast<uint4*>(dst + d * npad + c * 16) =
+        *reinterpret_cast<const uint4*>(tile + d * kKvRows + c * 16);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quant_v_rotated(int B, int Nkv, int Hkv, int D, BNHD v, QuantWorkspace ws,
+                                   int8_t* v8t, float* v_scale, cudaStream_t st) {
+  const int nK = (Nkv + kKvRows - 1) / kKvRows;
+  const dim3 grid(nK, B * Hkv);
+  switch (D) {
+    case 64: vrot_stats_kernel<64><<<grid, 256, 0, st>>>(v, Nkv, Hkv, nK, ws.vmax); break;
+    case 256: vrot_stats_kernel<256><<<grid, 256, 0, st>>>(v, Nkv, Hkv, nK, ws.vmax); break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int C = Hkv * D;
+  const int64_t cols = static_cast<int64_t>(B) * C;
+  kv_finalize_kernel<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+      B, Nkv, nK, C, false, nullptr, ws.vmax, nullptr, v_scale, ws.vfac, 127.0f);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  switch (D) {
+    case 64: vrot_quant_kernel<64><<<grid, 256, 0, st>>>(v, Nkv, Hkv, nK, ws.vfac, v8t); break;
+    case 256: vrot_quant_kernel<256><<<grid, 256, 0, st>>>(v, Nkv, Hkv, nK, ws.vfac, v8t); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 size_t quant_workspace_bytes(int B, int Nkv, int Hkv, int D) {
   const size_t nK = (static_cast<size_t>(Nkv) + kKvRows - 1) / kKvRows;
@@ -834,9 +985,9 @@ cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD
   const int tab_bytes = 2 * kKvRows * (rotary_dim / 2) * 2;
   const int smem1 = tab_bytes + kKvRows * D * 2;
   switch (D) {
-    case 64: e = launch_dyn(prep_stats_kernel<64>, grid1, 128, smem1, st, pa); break;
-    case 128: e = launch_dyn(prep_stats_kernel<128>, grid1, 128, smem1, st, pa); break;
-    case 256: e = launch_dyn(prep_stats_kernel<256>, grid1, 128, smem1, st, pa); break;
+    case 64: e = launch_dyn(prep_stats_kernel<64>, grid1, kPrepStatsThreads, smem1, st, pa); break;
+    case 128: e = launch_dyn(prep_stats_kernel<128>, grid1, kPrepStatsThreads, smem1, st, pa); break;
+    case 256: e = launch_dyn(prep_stats_kernel<256>, grid1, kPrepStatsThreads, smem1, st, pa); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -860,9 +1011,9 @@ cudaError_t launch_prep_quant(int B, int N, int Hq, int Hkv, int D, BNHD q, BNHD
   a.k_raw = true; a.kw = kw; a.eps = eps; a.rotary_dim = rotary_dim; a.cos_t = cos_t; a.sin_t = sin_t;
   const unsigned g2 = static_cast<unsigned>(a.nk_blocks + a.nv_blocks);
   switch (D) {   // dynamic shared memory: the staged RoPE tables of a raw-K block
-    case 64: return launch_dyn(quant_kernel<64>, g2, 128, tab_bytes, st, a);
-    case 128: return launch_dyn(quant_kernel<128>, g2, 128, tab_bytes, st, a);
-    case 256: return launch_dyn(quant_kernel<256>, g2, 128, tab_bytes, st, a);
+    case 64: return launch_dyn(quant_kernel<64, true>, g2, 128, tab_bytes, st, a);
+    case 128: return launch_dyn(quant_kernel<128, true>, g2, 128, tab_bytes, st, a);
+    case 256: return launch_dyn(quant_kernel<256, true>, g2, 128, tab_bytes, st, a);
     default: return cudaErrorInvalidValue;
   }
 }

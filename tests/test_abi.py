@@ -215,3 +215,11 @@ def test_quant_k32_refuses_like_quant(lib):
                                FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == 5
     assert lib.qattn_quant_k32(1, 64, 64, 1, 1, 96, _view(), _view(), _view(), FAKE, FAKE, FAKE,
                                FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 4
+
+
+def test_int8v_refusals(lib):
+    assert lib.qattn_fwd_int8v(1, 128, 128, 2, 2, 128, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, 0.0,
+                               FAKE, FAKE, None) == 4          # D must be 256
+    assert lib.qattn_quant_v_rotated(1, 128, 2, 128, _view(), FAKE, FAKE, FAKE, 1 << 20, None) == 4
+    assert lib.qattn_quant_v_rotated(1, 128, 2, 256, _view(), None, FAKE, FAKE, 1 << 20, None) == 1
+    assert lib.qattn_quant_v_rotated(1, 128, 2, 256, _view(), FAKE, FAKE, FAKE, 16, None) == 5

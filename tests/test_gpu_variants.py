@@ -121,3 +121,55 @@ def test_k32_scales_match_oracle(B, N, H, Hkv, D):
     exp, _, _ = O.attention(ref["q8"], ref["q_scale"], k8, ks, ref["v8t"], ref["v_scale"], N,
                             k_scale_mode=2)
     assert_out_close(host(out), exp, "k32")
+
+
+# --------------------------------------------------------------------- rotated INT8 V
+def _int8v(pipe, v_dev, w, mode):
+    nk = -(-w.Nkv // 64)
+    v8t = torch.empty((w.B, w.Hkv, w.D, 64 * nk), dtype=torch.int8, device=DEV)
+    vs = torch.empty((w.B, w.Hkv, w.D), dtype=torch.float32, device=DEV)
+    qa.qattn_quant_v_rotated(w.B, w.Nkv, w.Hkv, w.D, v_dev, v8t, vs, pipe.ws)
+    out = torch.empty((w.B, w.Nq, w.Hq, w.D), dtype=torch.bfloat16, device=DEV)
+    qa.qattn_fwd_int8v(w.B, w.Nq, w.Nkv, w.Hq, w.Hkv, w.D, pipe.q8, pipe.q_scale, pipe.k8,
+                       pipe.k_scale, mode, v8t, vs, 0.0, out, pipe.dev_err)
+    qa.qattn_check(pipe.dev_err)
+    return host(v8t), host(vs), host(out)
+
+
+@pytest.mark.parametrize("Nq,Nkv,Hq,Hkv,D", [(200, 1000, 16, 4, 256), (130, 97, 8, 2, 256),
+                                             (64, 3000, 4, 1, 256)])
+def test_int8v_rotated_gqa_matches_oracle(Nq, Nkv, Hq, Hkv, D):
+    w = synth.make("gqa_chunk", Nq=Nq, Nkv=Nkv, Hq=Hq, Hkv=Hkv, D=D, seed=Nq + Nkv + 7)
+    pipe = run_pipeline(w)
+    ref = oracle_full(w)
+    _, _, v, _keep = inputs_on_device(w)
+    v8t, vs, out = _int8v(pipe, v, w, 1)
+    exp_v8t, exp_vs = O.quant_v_rotated(w.v)
+    assert np.array_equal(v8t, exp_v8t) and np.array_equal(vs, exp_vs)
+    exp, _, _ = O.attention(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], exp_v8t, exp_vs,
+                            w.Nkv, k_scale_mode=1, pv="int8v")
+    assert_out_close(out, exp, "rotated int8 V")
+
+
+def test_int8v_with_block_k_scales_and_d64_quantizer():
+    # D = 256 attention with per-64-row K scales (the standard quantizer), and the
+    # D = 64 rotated V quantizer on its own
+    w = synth.custom(5151, 1, 300, 4, 256, rope=True, Hkv=2)
+    pipe = run_pipeline(w)
+    ref = oracle_full(w)
+    _, _, v, _keep = inputs_on_device(w)
+    v8t, vs, out = _int8v(pipe, v, w, 0)
+    exp_v8t, exp_vs = O.quant_v_rotated(w.v)
+    assert np.array_equal(v8t, exp_v8t) and np.array_equal(vs, exp_vs)
+    exp, _, _ = O.attention(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], exp_v8t, exp_vs,
+                            w.Nkv, pv="int8v")
+    assert_out_close(out, exp, "rotated int8 V, block K scales")
+    w64 = synth.custom(5152, 2, 150, 2, 64, rope=False)
+    v64 = dev_bf16(w64.v)
+    ws = torch.empty(qa.qattn_quant_workspace_bytes(2, 150, 2, 64), dtype=torch.uint8, device=DEV)
+    v8t64 = torch.empty((2, 2, 64, 192), dtype=torch.int8, device=DEV)
+    vs64 = torch.empty((2, 2, 64), dtype=torch.float32, device=DEV)
+    qa.qattn_quant_v_rotated(2, 150, 2, 64, v64, v8t64, vs64, ws)
+    torch.cuda.synchronize()
+    e8, es = O.quant_v_rotated(w64.v)
+    assert np.array_equal(host(v8t64), e8) and np.array_equal(host(vs64), es)

@@ -192,3 +192,54 @@ def test_kcache_attention_tracks_unrotated_fp64_attention():
                             cache["v16"][..., :150], None, 150, k_scale_mode=1, pv="fp16")
     cos_bad = float(_f(bad).ravel() @ ref.ravel() / np.linalg.norm(_f(bad)) / np.linalg.norm(ref))
     assert cos_bad < 0.95
+
+
+def _sylvester(n):
+    h = np.array([[1.0]])
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def test_quant_v_rotated_round_trip_and_channel_maxima():
+    rng = np.random.default_rng(28)
+    b, n, h, d = 1, 90, 2, 64
+    v = rng.standard_normal((b, n, h, d)).astype(np.float32)
+    v[:, :, :, 3] *= 8.0                                   # an outlier channel
+    vb = _bf(v)
+    v8t, vs = O.quant_v_rotated(vb)
+    assert v8t.shape == (b, h, d, 128) and v8t.dtype == np.int8 and vs.shape == (b, h, d)
+    assert not v8t[..., n:].any()
+    # every channel's maximum code is +-127 (amax maps to 127)
+    assert np.all(np.abs(v8t[..., :n]).max(axis=-1) == 127)
+    # decode, rotate back with an independent dense Sylvester matrix: V within half a
+    # scale step of the rotation of each channel
+    vr_dec = v8t[..., :n].astype(np.float64) * vs[..., None]          # [B,H,D,N]
+    back = np.einsum("bhdn,de->bnhe", vr_dec, _sylvester(d) / math.sqrt(d))
+    err = np.abs(back - _f(vb))
+    bound = 0.5 * np.sqrt(np.sum(vs.astype(np.float64) ** 2, axis=-1)) * 1.0001   # per (b, h)
+    assert np.all(err <= bound[:, None, :, None])
+
+
+def test_int8v_output_is_the_inverse_rotation_of_the_fp16_path():
+    # with the codes as FP16 V in the FP16 path (exact: |code| <= 127) and unit-power
+    # scales, the rotated-V output must be bf16(H (o * s) / sqrt(D)) of the FP16
+    # path's o; an independent dense Sylvester matrix stands in for the oracle's FWHT
+    rng = np.random.default_rng(29)
+    d, nq, nkv = 64, 20, 100
+    q8 = rng.integers(-127, 128, (1, 1, nq, d)).astype(np.int8)
+    qs = (0.01 + 0.01 * rng.random((1, 1, 4))).astype(np.float32)
+    k8 = rng.integers(-127, 128, (1, 1, nkv, d)).astype(np.int8)
+    ks = (0.01 + 0.01 * rng.random((1, 1, 2))).astype(np.float32)
+    v8t = np.zeros((1, 1, d, 128), np.int8)
+    v8t[..., :nkv] = rng.integers(-127, 128, (1, 1, d, nkv))
+    s = (2.0 ** rng.integers(-4, 3, (1, 1, d))).astype(np.float32)
+    v16 = f16_bits_from_f32(v8t.astype(np.float32))
+    o16, _, _ = O.attention(q8, qs, k8, ks, v16, None, nkv, pv="fp16")
+    o8, _, _ = O.attention(q8, qs, k8, ks, v8t, s, nkv, pv="int8v")
+    pre = _f(o16)[0, :, 0] * s[0, 0].astype(np.float64)               # [nq, d]
+    ref = (pre @ _sylvester(d).T) / math.sqrt(d)
+    got = _f(o8)[0, :, 0]
+    assert np.max(np.abs(got - ref)) <= 4 * 2.0 ** -8 * np.max(np.abs(ref))
+    wrong = (pre @ _sylvester(d)[::-1].T) / math.sqrt(d)               # a permuted transform
+    assert np.max(np.abs(got - wrong)) > 0.1 * np.max(np.abs(ref))

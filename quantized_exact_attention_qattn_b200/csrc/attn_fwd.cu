@@ -372,12 +372,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp >= C::SOFTMAX_WARP0) {
     if constexpr (C::HALVES) {
-      // ================================================================ softmax, D = 128
+      // ================================================================ softmax, two threads per row
       // Eight warps per query tile, two threads per row of the same warp.  Warp
       // slot s = 0..7 of tile i covers lanes 32 (s % 4) + 16 (s / 4) .. +15 (its
       // sub-partition's quadrant); of lane r's two threads, the first (thread r)
-      // owns keys 0-31 of each tile and O columns 0-63, the second (thread r + 16)
-      // keys 32-63 and O columns 64-127 (16x32bx2 accesses).  The row's tile
+      // owns keys 0-31 of each tile and O columns 0 .. D/2-1, the second (thread
+      // r + 16) keys 32-63 and O columns D/2 .. D-1 (16x32bx2 accesses).  The row's tile
       // maximum is one shuffle between the two; each keeps its own partial
       // denominator, added at the end.
       const int slot = warp - C::SOFTMAX_WARP0;

@@ -7,8 +7,8 @@ in-flight copies and MMAs and returns, and qattn_check reports QATTN_ERR_TIMEOUT
 with the error bits.  The CUDA context stays usable: the next call, with the hook
 off, gives exactly the output of the call before the failure.  Covered for the
 layout with one softmax warpgroup per query tile (D=128, two query tiles with Q
-in tensor memory; D=64, three query tiles with Q in shared memory) and the split
-layout with two warpgroups per query tile (D=256, per-token K scales).
+in tensor memory; D=64, three query tiles with Q in shared memory) and the
+layout with two threads per query row in eight warps (D=256, per-token K scales).
 """
 import pytest
 import torch

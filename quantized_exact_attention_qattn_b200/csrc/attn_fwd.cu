@@ -21,10 +21,11 @@
 //               scores, the online-softmax update, tcgen05.st of its 64
 //               probabilities, the O rescale of its row (only in warps where some
 //               row's maximum moved, after the previous P.V completed), and the
-//               final normalisation + BF16 store.  S is preloaded with the bits
-//               of 1.5 * 2^23 and QK accumulates onto them, so the scores read
-//               back as FP32 with one packed subtract per pair and no conversion;
-//               the reader re-preloads S and releases it to the next QK at once.
+//               final normalisation + BF16 store.  Each QK starts with a BF16
+//               MMA that writes the FP32 bias 1.53125 * 2^23 into S and the INT8
+//               MMAs accumulate onto its bits, so the scores read back as FP32
+//               with one packed subtract per pair and no conversion, and the
+//               reader releases S to the next QK right after its load.
 //               D = 256: eight warps per query tile, two threads per row of the
 //               same warp (16x32bx2 accesses): each owns 32 of the tile's keys and
 //               half of the O columns, the row maximum is one shuffle between the
@@ -88,13 +89,18 @@ struct Cfg {
   // for D = 256 (and D = 128 when QATTN_D128_HALVES is set), two threads per row
   // inside one warp (16x32bx2 tensor-memory accesses), eight warps per query tile
   static constexpr bool HALVES = (D == 256) || ((D == 128) && (QATTN_D128_HALVES != 0));
-  // D <= 128: S is preloaded with the bits of 1.5 * 2^23 and QK accumulates onto
-  // them; D = 256: QK overwrites S and the warps convert with I2F
+  // D <= 128: each QK first writes the FP32 bias kSBias into S (a BF16 MMA) and
+  // the INT8 steps accumulate onto its bits; D = 256: QK overwrites S and the
+  // warps convert with I2F
   static constexpr bool S_PRELOAD = (D <= 128);
   static constexpr int SM_WARPS = (HALVES ? 8 : 4) * NQT;           // softmax warps
   static constexpr int ARRIVALS = HALVES ? 8 : 4;                   // softmax warps per query tile
   static constexpr int SMEM_VST = SMEM_V + STAGES * V_BYTES;
-  static constexpr int SMEM_KS = SMEM_VST + STAGES * VST_BYTES;     // float [softmax warps][64]
+  // D <= 128: the constant BF16 operand tile of the score-bias MMA (128 rows of 128
+  // bytes, 128-byte swizzle; every element 896.0, so the layout does not matter)
+  static constexpr int SMEM_CB = SMEM_VST + STAGES * VST_BYTES;
+  static constexpr int CB_BYTES = S_PRELOAD ? BM * 128 : 0;
+  static constexpr int SMEM_KS = SMEM_CB + CB_BYTES;               // float [softmax warps][64]
   static constexpr int SMEM_BAR = SMEM_KS + SM_WARPS * BN * 4;
   static constexpr int N_BARS = 1 + 2 * STAGES + 8 * NQT + (PV == 2 ? STAGES : 0);
   static constexpr int SMEM_BYTES = SMEM_BAR + N_BARS * 8 + 16;
@@ -111,6 +117,7 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(Q_COL + (Q_TMEM ? NQT * (D / 4) : 0) <= TMEM_COLS, "tensor memory budget");
   static constexpr uint32_t IDESC_QK = instr_desc(2, 1, BM, BN);   // s8 x s8 -> s32
+  static constexpr uint32_t IDESC_SB = instr_desc(1, 1, BM, BN);   // bf16 x bf16 -> f32 (score bias)
   // e4m3 x e4m3 -> f32 (kind::f8f6f4) or f16 x f16 -> f32 (kind::f16): format code 0 both
   static constexpr uint32_t IDESC_PV = instr_desc(1, 0, BM, D);
 };
@@ -161,7 +168,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // and every waiter waits for every phase in order.  Every other barrier's next
   // phase depends on its waiter having passed.
   uint64_t* s_full = kv_empty + C::STAGES;   // MMA -> softmax: S_i(t) in TMEM
-  uint64_t* s_free = s_full + NQT;           // softmax -> MMA: S_i read and reset
+  uint64_t* s_free = s_full + NQT;           // softmax -> MMA: S_i read
   uint64_t* p_full = s_free + NQT;           // [NQT][2] softmax -> MMA: P_i(t) written, O_i rescaled
   uint64_t* pv_done = p_full + 2 * NQT;      // [NQT][2] MMA -> softmax: PV_i(t) done
   uint64_t* drain = pv_done + 2 * NQT;
@@ -204,6 +211,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if constexpr (PV == 2)
       for (int s = 0; s < C::STAGES; ++s) mbar_init(v_ready + s, 2);   // two converter warps
     fence_barrier_init();
+  }
+  if constexpr (C::S_PRELOAD) {   // operand tile of the score-bias MMA, read by the tensor core
+    uint32_t* cb = reinterpret_cast<uint32_t*>(smem + C::SMEM_CB);
+    for (int i = threadIdx.x; i < C::CB_BYTES / 4; i += C::THREADS) cb[i] = kSBiasRootBf16x2;
+    fence_proxy_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
@@ -267,13 +279,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t sV = smem_u32(smem + C::SMEM_V);
       const uint32_t tS = tmem + C::S_COL + i * BN;
       const uint32_t tO = tmem + C::O_COL + i * D;
+      const uint64_t cbd = smem_desc(smem_u32(smem + C::SMEM_CB), 8 * 128, 2u);
       auto issue_qk = [&](int s) {
+        // D <= 128: S <- kSBias first (overwrite), the INT8 steps then accumulate onto it
+        if constexpr (C::S_PRELOAD) mma_f16_ss(tS, cbd, cbd, C::IDESC_SB, 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          // D = 256: the first K step overwrites S; D <= 128: onto the kMagic bits
+          // D = 256: the first K step overwrites S; D <= 128: onto the kSBias bits
           const uint32_t acc = (!C::S_PRELOAD && kk == 0) ? 0u : 1u;
           if constexpr (C::Q_TMEM)   // Q_i row r in lane r, 4 bytes per column, 8 columns per K step
             mma_i8_ts(tS, tmem + C::Q_COL + i * (D / 4) + kk * 8, bd, C::IDESC_QK, acc);
@@ -439,12 +454,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           else
             tmem_st16x2_x32<32>(tmem + lane_off + C::Q_COL + i * (D / 4), r);
         }
-        if constexpr (C::S_PRELOAD) {
-          // S accumulates onto the bits of kMagic (1.5 * 2^23), read back as FP32 it
-          // is exactly kMagic + S (|S| < 2^22)
-          tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);
-          tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
-        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -466,11 +475,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float x[32];                                    // keys 32 kh .. 32 kh + 31
           tmem_ld16x2_x32<32>(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
           tmem_wait_ld();
-          if constexpr (C::S_PRELOAD) {
-            tmem_st16x2_x16_bcast<32>(tS, 0x4B400000u);   // reset S for QK_i(t+1)
-            tmem_st16x2_x16_bcast<32>(tS + 16, 0x4B400000u);
-            tmem_wait_st();
-          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + i);
@@ -478,7 +482,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
           }
-          constexpr float kBias = C::S_PRELOAD ? kMagic : 0.0f;
+          constexpr float kBias = C::S_PRELOAD ? kSBias : 0.0f;
           if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kBias);
           const bool last = (t == nK - 1);
           const int k0 = kh * 32;                         // first key of this half
@@ -502,7 +506,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if constexpr (C::S_PRELOAD) {
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
-                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
                 x[j] = sj.x;
                 x[j + 1] = sj.y;
               }
@@ -523,7 +527,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if constexpr (C::S_PRELOAD) {
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
-                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
                 x[j] = sj.x;
                 x[j + 1] = sj.y;
               }
@@ -716,17 +720,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           __syncwarp();
           if (lane == 0) mbar_arrive(q_ready + wg);
         }
-        // S accumulates onto the bits of kMagic (1.5 * 2^23): the INT32 sum kMagic + S
-        // read back as FP32 is exactly kMagic + S (|S| < 2^22), so no integer-to-float
-        // conversion is needed.
-        uint32_t magic[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) magic[j] = 0x4B400000u;
-        reset_s(tS, magic);
-        tmem_wait_st();
-        tc_fence_before();
+        // S arrives as kSBias + S (the issuer's bias MMA precedes each QK), read back
+        // as FP32 exactly; one subtraction recovers S
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + wg);      // s_free phase t: QK_i(t) may accumulate
+        if (lane == 0) mbar_arrive(s_free + wg);      // s_free phase t: QK_i(t) may write S
         bool ok = true;
         for (int t = 0; ok && t < nK; ++t) {
           float ks_cur = ks_next;
@@ -741,15 +738,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float x[64];
           tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
           tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-          tmem_wait_ld();
-          reset_s(tS, magic);                             // reset S for QK_i(t+1)
-          // release S right away: the next QK is on this warp's critical path, the
-          // store latency is short next to the max tree it would otherwise follow
-          tmem_wait_st();                                 // the reset of S has landed
+          tmem_wait_ld();                                 // S is in registers: release it
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + wg);
-          if constexpr (DUMP) dump_scores<64>(p, b, h, qt, t, row, 0, x, kMagic);
+          if constexpr (DUMP) dump_scores<64>(p, b, h, qt, t, row, 0, x, kSBias);
           const bool last = (t == nK - 1);
           float mn;
           float2 a2, nb2;
@@ -771,12 +764,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const float xmax = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
-              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
               x[j] = sj.x;
               x[j + 1] = sj.y;
             }
             const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-            const float smax = __fmul_rn(__fsub_rn(xmax, kMagic), a);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kSBias), a);
             mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
             a2 = make_float2(a, a);
             nb2 = make_float2(-mn, -mn);
@@ -792,7 +785,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // (every lane reads the same address: a broadcast, no bank conflict)
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
-              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kMagic, -kMagic));
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
               x[j] = sj.x;
               x[j + 1] = sj.y;
             }

@@ -281,8 +281,8 @@ qattn_status qattn_fwd_int8v(int B, int Nq, int Nkv, int Hq, int Hkv, int D,
  * ("INT8 QK And Score Domain"), for bit-exact checks of the path qattn_fwd runs.
  * This launches qattn_fwd's own kernel on the whole problem (same operands, same
  * TMA copies, same tcgen05 kind::i8 MMAs with Q read from tensor memory at D 128
- * and 256 and from shared memory at D 64, same score-bias MMA at D <= 128 and
- * integer-to-float conversion at D 256), built with one addition: when the softmax
+ * and 256 and from shared memory at D 64, same score-bias MMA and recovery of the
+ * INT32 value), built with one addition: when the softmax
  * warps have recovered the scores of a requested tile from tensor memory, they
  * also copy them out.  `out` receives the attention output as from qattn_fwd.
  *   tiles    int32 [n_tiles][4] = (b, h, q_tile, k_tile) (device, 16-byte

@@ -41,8 +41,7 @@ struct FwdParams {
 // Score copy-out of the debug build of the mainloop (qattn_scores).  The thread
 // owning query row `row` holds NCOL consecutive scores of key tile t, starting at
 // column col0, as the softmax reads them: x[j] - bias is the exact INT32 score
-// (bias = kSBias where S accumulated onto the bias MMA's output, 0 where it was
-// converted).  Every slot whose request names (b, h, qt, t) receives them; the
+// (bias = kSBias, the output of the bias MMA that the scores accumulate onto).  Every slot whose request names (b, h, qt, t) receives them; the
 // warp's lanes scan the request list 32 entries at a time.
 template <int NCOL>
 __device__ __forceinline__ void dump_scores(const FwdParams& p, int b, int h, int qt, int t,
@@ -76,14 +75,15 @@ __device__ __forceinline__ void dump_scores(const FwdParams& p, int b, int h, in
 #endif
 constexpr int kPolyPer8 = QATTN_POLY_PER8;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: x + kMagic rounds x to an integer
-// Score bias (D <= 128).  Before each QK the tensor core writes kSBias = 16 * 896^2
-// = 1.53125 * 2^23 into S (one BF16 MMA, K = 16, every operand element 896.0, an
-// exact FP32 sum), and the INT8 MMAs then add the INT32 score S onto those bits.
-// The mantissa field 0x440000 + S stays inside [0, 2^23) for -4456448 <= S <
-// 3932160 (|S| <= 128 * 127 * 128 here), so the word read back as FP32 is
-// exactly kSBias + S: one subtraction recovers S, no integer-to-float conversion.
-constexpr float kSBias = 12845056.0f;
-constexpr uint32_t kSBiasRootBf16x2 = 0x44604460u;   // two BF16 896.0
+// Score bias.  Before each QK the tensor core writes kSBias = 16 * 888^2 =
+// 12616704 = 2^23 + 0x408400 into S (one BF16 MMA, K = 16, every operand element
+// 888.0, an exact FP32 sum), and the INT8 MMAs then add the INT32 score S onto
+// those bits.  The mantissa field 0x408400 + S stays inside [0, 2^23) for
+// -4228096 <= S < 4160512, which holds every score of INT8 codes in [-127, 127]
+// up to D = 256 (|S| <= 256 * 127 * 127 = 4129024), so the word read back as FP32
+// is exactly kSBias + S: one subtraction recovers S, no integer-to-float conversion.
+constexpr float kSBias = 12616704.0f;
+constexpr uint32_t kSBiasRootBf16x2 = 0x445E445Eu;   // two BF16 888.0
 // 2^f on [-1/2, 1/2], degree 5, relative minimax (fit_exp2.py), max relative error
 // 2.3e-7 in FP32: about that of ex2.approx, so both paths round P to E4M3 alike.
 constexpr float kC0 = 1.000000119e+00f, kC1 = 6.931469440e-01f, kC2 = 2.402212024e-01f,

@@ -29,9 +29,7 @@
 //               D = 256: eight warps per query tile, two threads per row of the
 //               same warp (16x32bx2 accesses): each owns 32 of the tile's keys and
 //               half of the O columns, the row maximum is one shuffle between the
-//               two, and each keeps a partial denominator added at the end.  Here
-//               QK overwrites S and the warps convert their INT32 scores with I2F,
-//               which frees S for the next QK right after the load.
+//               two, and each keeps a partial denominator added at the end.
 // The query tiles' chains (two per CTA at D = 128, three at D = 64, where the
 // smaller O leaves TMEM room for a third) are independent, so while one warpgroup
 // runs the softmax of its tile the tensor core works for the others.  Every wait is
@@ -89,17 +87,14 @@ struct Cfg {
   // for D = 256 (and D = 128 when QATTN_D128_HALVES is set), two threads per row
   // inside one warp (16x32bx2 tensor-memory accesses), eight warps per query tile
   static constexpr bool HALVES = (D == 256) || ((D == 128) && (QATTN_D128_HALVES != 0));
-  // D <= 128: each QK first writes the FP32 bias kSBias into S (a BF16 MMA) and
-  // the INT8 steps accumulate onto its bits; D = 256: QK overwrites S and the
-  // warps convert with I2F
-  static constexpr bool S_PRELOAD = (D <= 128);
   static constexpr int SM_WARPS = (HALVES ? 8 : 4) * NQT;           // softmax warps
   static constexpr int ARRIVALS = HALVES ? 8 : 4;                   // softmax warps per query tile
   static constexpr int SMEM_VST = SMEM_V + STAGES * V_BYTES;
-  // D <= 128: the constant BF16 operand tile of the score-bias MMA (128 rows of 128
-  // bytes, 128-byte swizzle; every element 896.0, so the layout does not matter)
+  // The constant BF16 operand tile of the score-bias MMA that starts every QK (128
+  // rows of 128 bytes, 128-byte swizzle; every element 888.0, so the layout does
+  // not matter)
   static constexpr int SMEM_CB = SMEM_VST + STAGES * VST_BYTES;
-  static constexpr int CB_BYTES = S_PRELOAD ? BM * 128 : 0;
+  static constexpr int CB_BYTES = BM * 128;
   static constexpr int SMEM_KS = SMEM_CB + CB_BYTES;               // float [softmax warps][64]
   static constexpr int SMEM_BAR = SMEM_KS + SM_WARPS * BN * 4;
   static constexpr int N_BARS = 1 + 2 * STAGES + 8 * NQT + (PV == 2 ? STAGES : 0);
@@ -212,7 +207,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int s = 0; s < C::STAGES; ++s) mbar_init(v_ready + s, 2);   // two converter warps
     fence_barrier_init();
   }
-  if constexpr (C::S_PRELOAD) {   // operand tile of the score-bias MMA, read by the tensor core
+  {   // operand tile of the score-bias MMA, read by the tensor core
     uint32_t* cb = reinterpret_cast<uint32_t*>(smem + C::SMEM_CB);
     for (int i = threadIdx.x; i < C::CB_BYTES / 4; i += C::THREADS) cb[i] = kSBiasRootBf16x2;
     fence_proxy_async_smem();
@@ -281,20 +276,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t tO = tmem + C::O_COL + i * D;
       const uint64_t cbd = smem_desc(smem_u32(smem + C::SMEM_CB), 8 * 128, 2u);
       auto issue_qk = [&](int s) {
-        // D <= 128: S <- kSBias first (overwrite), the INT8 steps then accumulate onto it
-        if constexpr (C::S_PRELOAD) mma_f16_ss(tS, cbd, cbd, C::IDESC_SB, 0u);
+        // S <- kSBias first (overwrite), the INT8 steps then accumulate onto it
+        mma_f16_ss(tS, cbd, cbd, C::IDESC_SB, 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const int ch = (kk * 32) / C::KCH, off = (kk * 32) % C::KCH;
           const uint64_t bd = smem_desc(sK + s * C::K_BYTES + ch * (BN * C::KCH) + off,
                                         8 * C::KCH, C::SW_QK);
-          // D = 256: the first K step overwrites S; D <= 128: onto the kSBias bits
-          const uint32_t acc = (!C::S_PRELOAD && kk == 0) ? 0u : 1u;
           if constexpr (C::Q_TMEM)   // Q_i row r in lane r, 4 bytes per column, 8 columns per K step
-            mma_i8_ts(tS, tmem + C::Q_COL + i * (D / 4) + kk * 8, bd, C::IDESC_QK, acc);
+            mma_i8_ts(tS, tmem + C::Q_COL + i * (D / 4) + kk * 8, bd, C::IDESC_QK, 1u);
           else
             mma_i8_ss(tS, smem_desc(sQ + ch * (BM * C::KCH) + off, 8 * C::KCH, C::SW_QK), bd,
-                      C::IDESC_QK, acc);
+                      C::IDESC_QK, 1u);
         }
         tc_commit(s_full + i);
       };
@@ -478,12 +471,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free + i);
-          if constexpr (!C::S_PRELOAD) {                  // INT32 scores to FP32: exact, |S| < 2^24
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = __int2float_rn(__float_as_int(x[j]));
-          }
-          constexpr float kBias = C::S_PRELOAD ? kSBias : 0.0f;
-          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kBias);
+          if constexpr (DUMP) dump_scores<32>(p, b, h, qt, t, row, kh * 32, x, kSBias);
           const bool last = (t == nK - 1);
           const int k0 = kh * 32;                         // first key of this half
           float mn;
@@ -503,16 +491,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
             float xmax = fmaxf(mq[0], mq[1]);
             xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 16));   // the row's other half
-            if constexpr (C::S_PRELOAD) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 2) {
-                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
-                x[j] = sj.x;
-                x[j + 1] = sj.y;
-              }
+            for (int j = 0; j < 32; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
             }
             const float a = __fmul_rn(__fmul_rn(qs, ks_cur), p.c);
-            const float smax = __fmul_rn(__fsub_rn(xmax, kBias), a);
+            const float smax = __fmul_rn(__fsub_rn(xmax, kSBias), a);
             mn = fmaxf(m, __fsub_rn(smax, kFp8Offset));
             a2 = make_float2(a, a);
             nb2 = make_float2(-mn, -mn);
@@ -524,13 +510,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             kss[2 * lane] = kpair.x;
             kss[2 * lane + 1] = kpair.y;
             __syncwarp();
-            if constexpr (C::S_PRELOAD) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 2) {
-                const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
-                x[j] = sj.x;
-                x[j + 1] = sj.y;
-              }
+            for (int j = 0; j < 32; j += 2) {
+              const float2 sj = fadd2(make_float2(x[j], x[j + 1]), make_float2(-kSBias, -kSBias));
+              x[j] = sj.x;
+              x[j + 1] = sj.y;
             }
             const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;

@@ -129,23 +129,17 @@ __device__ __forceinline__ void exp_block(float (&x)[N], float2 a2, float2 nb2) 
   }
 }
 
-// Per-token K scales.  kss holds the tile's scales k_j (shared memory, every lane
-// reads the same addresses), qs2 = (q_scale, q_scale), c2 = (c, c); the score
-// scale of key j is A_j = (q_scale * k_j) * c, formed two keys at a time.
-__device__ __forceinline__ float2 kt_scale_pair(const float* kss, int j, float2 qs2, float2 c2) {
-  const float2 k2 = *reinterpret_cast<const float2*>(kss + j);
-  return fmul2(fmul2(qs2, k2), c2);
-}
-
-// max_j S_j * A_j over all N keys (every key valid), four independent chains.
+// Per-token K scales.  The warp stages the tile's score scales A_j = (q_scale *
+// k_j) * c in shared memory (q_scale is the same for all rows of a warp); every
+// lane reads the same addresses, a broadcast.  max_j S_j * A_j over all N keys
+// (every key valid), four independent chains.
 template <int N>
-__device__ __forceinline__ float kt_tile_max(const float (&x)[N], const float* kss, float2 qs2,
-                                             float2 c2) {
+__device__ __forceinline__ float kt_tile_max(const float (&x)[N], const float* as) {
   float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int j = 0; j < N; j += 4) {
-    const float2 s01 = fmul2(make_float2(x[j], x[j + 1]), kt_scale_pair(kss, j, qs2, c2));
-    const float2 s23 = fmul2(make_float2(x[j + 2], x[j + 3]), kt_scale_pair(kss, j + 2, qs2, c2));
+    const float2 s01 = fmul2(make_float2(x[j], x[j + 1]), *reinterpret_cast<const float2*>(as + j));
+    const float2 s23 = fmul2(make_float2(x[j + 2], x[j + 3]), *reinterpret_cast<const float2*>(as + j + 2));
     const int q = (j / 4) & 1;
     mq[q] = fmax3(mq[q], s01.x, s01.y);
     mq[2 + q] = fmax3(mq[2 + q], s23.x, s23.y);
@@ -155,14 +149,13 @@ __device__ __forceinline__ float kt_tile_max(const float (&x)[N], const float* k
 
 // x[j] holds the exact FP32 score S_j; p_j = 2^fma(S_j, A_j, -mn), columns J .. END-1.
 template <int J, int END, int N>
-__device__ __forceinline__ void exp_block_kt(float (&x)[N], const float* kss, float2 qs2,
-                                             float2 c2, float2 nb2) {
+__device__ __forceinline__ void exp_block_kt(float (&x)[N], const float* as, float2 nb2) {
   if constexpr (J < END) {
-    const float2 t = ffma2(make_float2(x[J], x[J + 1]), kt_scale_pair(kss, J, qs2, c2), nb2);
+    const float2 t = ffma2(make_float2(x[J], x[J + 1]), *reinterpret_cast<const float2*>(as + J), nb2);
     const float2 e = exp2_pair<J>(t);
     x[J] = e.x;
     x[J + 1] = e.y;
-    exp_block_kt<J + 2, END>(x, kss, qs2, c2, nb2);
+    exp_block_kt<J + 2, END>(x, as, nb2);
   }
 }
 

@@ -151,7 +151,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token K scales
+  float* ks_stage = reinterpret_cast<float*>(smem + C::SMEM_KS);   // per-token score scales A_j
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
@@ -503,12 +503,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             a2 = make_float2(a, a);
             nb2 = make_float2(-mn, -mn);
           } else {
-            // per-token K scales: the warp stages the tile's 64 scales (two per lane);
-            // each half reads its own 32
+            // per-token K scales: the warp stages the tile's 64 score scales
+            // A_j = (q_scale * k_j) * c (two per lane); each half reads its own 32
             const int nv = last ? last_valid : BN;
             float* kss = ks_stage + slot * BN;
-            kss[2 * lane] = kpair.x;
-            kss[2 * lane + 1] = kpair.y;
+            *reinterpret_cast<float2*>(kss + 2 * lane) =
+                fmul2(fmul2(make_float2(qs, qs), kpair), make_float2(p.c, p.c));
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -516,14 +516,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               x[j] = sj.x;
               x[j + 1] = sj.y;
             }
-            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;
             if (!last) {
-              smx = kt_tile_max<32>(x, kss + k0, qs2, c2);
+              smx = kt_tile_max<32>(x, kss + k0);
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (k0 + j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[k0 + j]), p.c)));
+                if (k0 + j < nv) smx = fmaxf(smx, __fmul_rn(x[j], kss[k0 + j]));
             }
             smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, 16));
             mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
@@ -533,8 +532,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if constexpr (KMODE == 0) {
             exp_block<0, 32>(x, a2, nb2);
           } else {
-            exp_block_kt<0, 32>(x, ks_stage + slot * BN + k0, make_float2(qs, qs),
-                                make_float2(p.c, p.c), nb2);
+            exp_block_kt<0, 32>(x, ks_stage + slot * BN + k0, nb2);
             __syncwarp();                                 // kss is rewritten next tile
             if (last) {
 #pragma unroll
@@ -759,12 +757,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             nb2 = make_float2(-mn, -mn);
           } else {
             // per-token K scales: A_j = (q_scale * k_scale_j) * c; the exponent is
-            // fma(S_j, A_j, -mn).  The warp stages the tile's 64 scales in shared
-            // memory (two per lane, one load each) and every thread keeps A_j.
+            // fma(S_j, A_j, -mn).  The warp stages the tile's 64 score scales A_j in
+            // shared memory (two per lane, from the K scales fetched a tile ago).
             const int nv = last ? last_valid : BN;
             float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
-            kss[2 * lane] = kpair.x;                      // this tile's scales, fetched a tile ago
-            kss[2 * lane + 1] = kpair.y;
+            *reinterpret_cast<float2*>(kss + 2 * lane) =
+                fmul2(fmul2(make_float2(qs, qs), kpair), make_float2(p.c, p.c));
             __syncwarp();
             // (every lane reads the same address: a broadcast, no bank conflict)
 #pragma unroll
@@ -773,14 +771,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               x[j] = sj.x;
               x[j + 1] = sj.y;
             }
-            const float2 qs2 = make_float2(qs, qs), c2 = make_float2(p.c, p.c);
             float smx = -INFINITY;
             if (!last) {
-              smx = kt_tile_max<64>(x, kss, qs2, c2);
+              smx = kt_tile_max<64>(x, kss);
             } else {
 #pragma unroll
               for (int j = 0; j < 64; ++j)
-                if (j < nv) smx = fmaxf(smx, __fmul_rn(x[j], __fmul_rn(__fmul_rn(qs, kss[j]), p.c)));
+                if (j < nv) smx = fmaxf(smx, __fmul_rn(x[j], kss[j]));
             }
             mn = fmaxf(m, __fsub_rn(smx, kFp8Offset));
             nb2 = make_float2(-mn, -mn);
@@ -789,8 +786,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if constexpr (KMODE == 0) {
             exp_block<0, 64>(x, a2, nb2);
           } else {
-            exp_block_kt<0, 64>(x, ks_stage + (warp - C::SOFTMAX_WARP0) * BN, make_float2(qs, qs),
-                                make_float2(p.c, p.c), nb2);
+            exp_block_kt<0, 64>(x, ks_stage + (warp - C::SOFTMAX_WARP0) * BN, nb2);
             __syncwarp();                                 // kss is rewritten next tile
             if (last) {
 #pragma unroll

@@ -410,19 +410,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
         // per-key scales: lane l holds those of tokens 2l, 2l+1 of a tile (0 past the
         // end): their own (mode 1) or their 32-row group's (mode 2)
-        auto load_kpair = [&](int tt) {
+        // The loads are issued a tile ahead into raw registers (predicated, nothing
+        // depends on them until the next tile stages its scales): a conversion right
+        // after the load would stall the warp for the load's whole latency.
+        auto load_kraw = [&](int tt) {
+          uint32_t a = 0, b = 0;
           if constexpr (KMODE == 2) {
             const int g = 2 * tt + (lane >> 4);
-            const float v = g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
-            return make_float2(v, v);
+            if (g < n_groups32) a = __float_as_uint(__ldg(ks32 + g));
           } else {
             const int j = tt * BN + 2 * lane;
-            return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
-                               j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+            const unsigned short* k16 = reinterpret_cast<const unsigned short*>(ks16);
+            if (j < p.Nkv) a = __ldg(k16 + j);
+            if (j + 1 < p.Nkv) b = __ldg(k16 + j + 1);
+          }
+          return make_uint2(a, b);
+        };
+        auto kraw_pair = [&](uint2 r) {
+          if constexpr (KMODE == 2) {
+            return make_float2(__uint_as_float(r.x), __uint_as_float(r.x));
+          } else {
+            return make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(r.x))),
+                               __half2float(__ushort_as_half(static_cast<unsigned short>(r.y))));
           }
         };
-        float2 kpair_next = make_float2(0.0f, 0.0f);
-        if constexpr (KMODE != 0) kpair_next = load_kpair(0);
+        uint2 kraw_next = make_uint2(0u, 0u);
+        if constexpr (KMODE != 0) kraw_next = load_kraw(0);
         {   // this thread's D/2 bytes of its Q row into tensor memory (D/8 columns)
           const int n = qt * BM + row;
           constexpr int QW = D / 8;                       // 32-bit words per thread
@@ -458,9 +471,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int t = 0; ok && t < nK; ++t) {
           const float ks_cur = ks_next;
           if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
-          const float2 kpair = kpair_next;
+          const uint2 kraw = kraw_next;
           if constexpr (KMODE != 0) {
-            if (t + 1 < nK) kpair_next = load_kpair(t + 1);
+            if (t + 1 < nK) kraw_next = load_kraw(t + 1);
           }
           ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, t & 1, abort, p.dev_err, kErrTimeoutS));
           if (!ok) break;
@@ -508,7 +521,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int nv = last ? last_valid : BN;
             float* kss = ks_stage + slot * BN;
             *reinterpret_cast<float2*>(kss + 2 * lane) =
-                fmul2(fmul2(make_float2(qs, qs), kpair), make_float2(p.c, p.c));
+                fmul2(fmul2(make_float2(qs, qs), kraw_pair(kraw)), make_float2(p.c, p.c));
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -681,19 +694,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         float ks_next = (KMODE == 0) ? ks32[0] : 0.0f;
         // per-key scales: lane l holds those of tokens 2l, 2l+1 of a tile (0 past the
         // end): their own (mode 1) or their 32-row group's (mode 2)
-        auto load_kpair = [&](int tt) {
+        // The loads are issued a tile ahead into raw registers (predicated, nothing
+        // depends on them until the next tile stages its scales): a conversion right
+        // after the load would stall the warp for the load's whole latency.
+        auto load_kraw = [&](int tt) {
+          uint32_t a = 0, b = 0;
           if constexpr (KMODE == 2) {
             const int g = 2 * tt + (lane >> 4);
-            const float v = g < n_groups32 ? __ldg(ks32 + g) : 0.0f;
-            return make_float2(v, v);
+            if (g < n_groups32) a = __float_as_uint(__ldg(ks32 + g));
           } else {
             const int j = tt * BN + 2 * lane;
-            return make_float2(j < p.Nkv ? __half2float(__ldg(ks16 + j)) : 0.0f,
-                               j + 1 < p.Nkv ? __half2float(__ldg(ks16 + j + 1)) : 0.0f);
+            const unsigned short* k16 = reinterpret_cast<const unsigned short*>(ks16);
+            if (j < p.Nkv) a = __ldg(k16 + j);
+            if (j + 1 < p.Nkv) b = __ldg(k16 + j + 1);
+          }
+          return make_uint2(a, b);
+        };
+        auto kraw_pair = [&](uint2 r) {
+          if constexpr (KMODE == 2) {
+            return make_float2(__uint_as_float(r.x), __uint_as_float(r.x));
+          } else {
+            return make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(r.x))),
+                               __half2float(__ushort_as_half(static_cast<unsigned short>(r.y))));
           }
         };
-        float2 kpair_next = make_float2(0.0f, 0.0f);
-        if constexpr (KMODE != 0) kpair_next = load_kpair(0);
+        uint2 kraw_next = make_uint2(0u, 0u);
+        if constexpr (KMODE != 0) kraw_next = load_kraw(0);
         if constexpr (C::Q_TMEM) {   // this warp's rows of Q_i (D = 128: 32 columns)
           static_assert(!C::Q_TMEM || D == 128, "one 32-column store per row");
           store_q_row(p, bh, qt * BM + row, D, 0, tmem + lane_off + C::Q_COL + wg * (D / 4));
@@ -710,9 +736,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int t = 0; ok && t < nK; ++t) {
           float ks_cur = ks_next;
           if (KMODE == 0 && t + 1 < nK) ks_next = ks32[t + 1];   // prefetch next tile's scale
-          const float2 kpair = kpair_next;
+          const uint2 kraw = kraw_next;
           if constexpr (KMODE != 0) {
-            if (t + 1 < nK) kpair_next = load_kpair(t + 1);
+            if (t + 1 < nK) kraw_next = load_kraw(t + 1);
           }
           ok = __all_sync(0xffffffffu, mbar_wait(s_full + wg, t & 1, abort, p.dev_err, kErrTimeoutS));
           if (!ok) break;
@@ -762,7 +788,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int nv = last ? last_valid : BN;
             float* kss = ks_stage + (warp - C::SOFTMAX_WARP0) * BN;
             *reinterpret_cast<float2*>(kss + 2 * lane) =
-                fmul2(fmul2(make_float2(qs, qs), kpair), make_float2(p.c, p.c));
+                fmul2(fmul2(make_float2(qs, qs), kraw_pair(kraw)), make_float2(p.c, p.c));
             __syncwarp();
             // (every lane reads the same address: a broadcast, no bank conflict)
 #pragma unroll

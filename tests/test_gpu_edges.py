@@ -215,3 +215,26 @@ def test_repeat_calls_are_deterministic():
     a.run_fwd()
     a.check()
     assert torch.equal(first.view(torch.int16), a.out.view(torch.int16))
+
+
+@pytest.mark.parametrize("pos_offset,theta", [(0, 1e4), ((1 << 20) - 2048, 1e4),
+                                              ((1 << 24) - 2048, 1e4), ((1 << 24) - 2048, 5e5)])
+def test_rope_coefficients_wide_positions(pos_offset, theta):
+    # The BF16 RoPE coefficients the library derives on the device (FP64 frequency,
+    # angle, cos and sin, one rounding each; "Preparation" step 3) against the
+    # oracle's numpy FP64 tables, up to position 2^24.  Head h of every row holds a
+    # one-hot 1.0 at dim h and no norm is applied, so the prepared row carries
+    # cos_h(pos) at dim h and sin_h(pos) at dim h + R/2, exactly.
+    N, R, D = 2048, 96, 128
+    half = R // 2
+    x = np.zeros((1, N, half, D), np.uint16)
+    x[0, :, np.arange(half), np.arange(half)] = 0x3F80            # BF16 1.0
+    q = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(DEV)
+    pipe = qa.Pipeline(1, N, N, half, half, D, device=DEV)
+    pipe.run_prep(q, q, None, None, 1e-5, R, theta, pos_offset=pos_offset)
+    torch.cuda.synchronize()
+    got = host(pipe.qp)[0]                                         # [N, half, D] BF16 bits
+    cos_ref, sin_ref = O.rope_tables(N, R, theta, pos_offset)
+    h = np.arange(half)
+    assert np.array_equal(got[:, h, h], cos_ref)
+    assert np.array_equal(got[:, h, h + half], sin_ref)

@@ -80,3 +80,35 @@ def test_scores_requests_outside_the_problem_leave_slots_untouched():
     assert np.array_equal(s[0], s[5])
     for n in range(1, 5):
         assert (s[n] == SENTINEL).all(), tl[n]
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_scores_at_the_int8_extremes(D):
+    # Codes of +-127 in every lane give the largest |S| the quantizers can produce,
+    # D * 127^2 (4,129,024 at D = 256): the scores that the mainloop recovers from
+    # the bits of its score-bias MMA output stay exact at both ends of the range.
+    N, nq, nk = 192, 2, 3
+    rng = np.random.default_rng(D)
+    q8 = rng.choice(np.array([127, -127], np.int8), size=(1, 1, N, D))
+    k8 = rng.choice(np.array([127, -127], np.int8), size=(1, 1, N, D))
+    q8[0, 0, :40] = 127                         # rows of all +127 ...
+    q8[0, 0, 130:150] = -127                    # ... and of all -127
+    k8[0, 0, :20] = 127
+    k8[0, 0, 64:90] = -127
+    k8[0, 0, 150:170] = 127
+    pipe = qa.Pipeline(1, N, N, 1, 1, D, device=DEV)
+    pipe.q8.copy_(torch.from_numpy(q8))
+    pipe.k8.copy_(torch.from_numpy(k8))
+    pipe.q_scale.fill_(1.0 / 127)
+    pipe.k_scale.fill_(1.0 / 127)
+    codes = rng.integers(0, 256, size=tuple(pipe.v8t.shape), dtype=np.uint8) & 0x77   # finite E4M3
+    pipe.v8t.copy_(torch.from_numpy(codes))
+    pipe.v_scale.fill_(1.0)
+    pipe.run_fwd()
+    pipe.check()
+    tl = [(0, 0, qt, kt) for qt in range(nq) for kt in range(nk)]
+    s = hot_path_scores(pipe, tl)
+    assert s.min() == -D * 127 * 127 and s.max() == D * 127 * 127
+    for i, (_, _, qt, kt) in enumerate(tl):
+        assert_scores_tile(s[i], q8[0, 0, qt * 128:(qt + 1) * 128], k8[0, 0, kt * 64:(kt + 1) * 64],
+                           ("D", D, qt, kt))

@@ -189,19 +189,22 @@ __device__ __forceinline__ void rescale_rows(uint32_t tO, float o) {
 // threads 16-31 columns HALF .. 2 HALF-1), 32 columns at a time.
 template <int HALF>
 __device__ __forceinline__ void rescale_halves(uint32_t tO, float o) {
+  static_assert(HALF % 64 == 0, "64-column round trips");
 #pragma unroll 1
-  for (int c0 = 0; c0 < HALF; c0 += 32) {
-    uint32_t r[32];
-    tmem_ld16x2_x32<HALF>(tO + c0, r);
+  for (int c0 = 0; c0 < HALF; c0 += 64) {           // two 32-column loads per round trip
+    uint32_t r[64];
+    tmem_ld16x2_x32<HALF>(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld16x2_x32<HALF>(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
+    for (int j = 0; j < 64; j += 2) {
       const float2 v = fmul2(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
                              make_float2(o, o));
       r[j] = __float_as_uint(v.x);
       r[j + 1] = __float_as_uint(v.y);
     }
-    tmem_st16x2_x32<HALF>(tO + c0, r);
+    tmem_st16x2_x32<HALF>(tO + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_st16x2_x32<HALF>(tO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
   }
 }
 

@@ -22,7 +22,7 @@
 //               probabilities, the O rescale of its row (only in warps where some
 //               row's maximum moved, after the previous P.V completed), and the
 //               final normalisation + BF16 store.  Each QK starts with a BF16
-//               MMA that writes the FP32 bias 1.53125 * 2^23 into S and the INT8
+//               MMA that writes the FP32 bias kSBias = 16 * 888^2 into S and the INT8
 //               MMAs accumulate onto its bits, so the scores read back as FP32
 //               with one packed subtract per pair and no conversion, and the
 //               reader releases S to the next QK right after its load.

@@ -474,8 +474,10 @@ struct PrepStatsArgs {
 // Dynamic shared memory: tables 2 x 64 x R/2 BF16, then (K/V CTAs) 64 x D BF16.
 constexpr int kPrepStatsThreads = 256;
 
+// D <= 128: at most 64 registers (four CTAs per SM), so a CTA also fits beside an
+// attention CTA of another stream (the host pipeline overlaps the two)
 template <int D>
-__global__ void __launch_bounds__(kPrepStatsThreads) prep_stats_kernel(const PrepStatsArgs a) {
+__global__ void __launch_bounds__(kPrepStatsThreads, D <= 128 ? 4 : 1) prep_stats_kernel(const PrepStatsArgs a) {
   constexpr int L = D / 8, HPW = 32 / L;       // lanes per row, rows per warp
   constexpr int NW = kPrepStatsThreads / 32;
   constexpr int RPP = NW * HPW;                // rows per pass

@@ -55,10 +55,6 @@ using namespace attn;
 
 constexpr int BN = 64;    // keys per tile ("Online Softmax": 64-key tiles)
 
-#ifndef QATTN_D128_HALVES
-#define QATTN_D128_HALVES 0
-#endif
-
 // PV 0: FP8 E4M3 P and V (kind::f8f6f4), two P buffers of 16 columns per query
 // tile; PV 1: FP16 P and V (kind::f16), one P buffer of 32 columns (the same
 // tensor-memory columns) and V tiles of 64 keys x 2 bytes per dim row; PV 2 (D =
@@ -84,9 +80,9 @@ struct Cfg {
   static constexpr int SMEM_K = SMEM_Q + (Q_TMEM ? 0 : NQT * Q_BYTES);
   static constexpr int SMEM_V = SMEM_K + STAGES * K_BYTES;
   // Softmax layout: one thread per query row (one warpgroup per query tile), or,
-  // for D = 256 (and D = 128 when QATTN_D128_HALVES is set), two threads per row
-  // inside one warp (16x32bx2 tensor-memory accesses), eight warps per query tile
-  static constexpr bool HALVES = (D == 256) || ((D == 128) && (QATTN_D128_HALVES != 0));
+  // for D = 256, two threads per row inside one warp (16x32bx2 tensor-memory
+  // accesses), eight warps per query tile
+  static constexpr bool HALVES = (D == 256);
   static constexpr int SM_WARPS = (HALVES ? 8 : 4) * NQT;           // softmax warps
   static constexpr int ARRIVALS = HALVES ? 8 : 4;                   // softmax warps per query tile
   static constexpr int SMEM_VST = SMEM_V + STAGES * V_BYTES;
